@@ -1,0 +1,190 @@
+"""CPU oracle for block-sparse 3D-video attention -- test infrastructure.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  It wraps ``vsa_oracle.c`` (plain fp64 C, built
+with gcc into ``liborc.so`` beside it) through ctypes and shares no code with
+the CUDA library.  What each function follows is stated in ``vsa_oracle.c``.
+
+Classification of a tile pair from brute-force counts (the three tile kinds of
+"Sparse VideoGen: accelerating video diffusion attention on TPU", section
+"logical sparsity is not physical sparsity"): 0 empty when no (real query,
+key slot) pair is kept, 2 full when every such pair is kept (a kv tile holding
+padding is therefore never full), 1 boundary otherwise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from typing import Dict, Iterable, Optional, Sequence, Tuple
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "vsa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liborc.so")
+_lib = None
+
+
+class _Mask(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int32) for k in
+                ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
+                 "Tw", "To", "Ts", "Sw", "So", "Ss")]
+
+
+class _Grid(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_int32) for k in ("T", "H", "W", "bt", "bh", "bw")]
+
+
+def build_oracle(force: bool = False) -> str:
+    """Compile liborc.so with gcc (plain C, -O2, pthreads)."""
+    if force or not os.path.exists(_LIB_PATH) or \
+            os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-shared", "-fPIC",
+                               "-o", tmp, _SRC, "-lpthread", "-lm"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_oracle())
+        P = ctypes.POINTER
+        lib.orc_padded_tokens.restype = ctypes.c_int64
+        lib.orc_padded_tokens.argtypes = [P(_Grid)]
+        lib.orc_tile_major_order.restype = ctypes.c_int64
+        lib.orc_tile_major_order.argtypes = [P(_Grid), ctypes.c_int64, ctypes.c_void_p]
+        lib.orc_keep.restype = ctypes.c_int
+        lib.orc_keep.argtypes = [P(_Mask), P(_Grid), ctypes.c_int64, ctypes.c_int64]
+        lib.orc_keep_matrix.restype = ctypes.c_int
+        lib.orc_keep_matrix.argtypes = [P(_Mask), P(_Grid), ctypes.c_void_p]
+        lib.orc_attention_rows.restype = ctypes.c_int
+        lib.orc_attention_rows.argtypes = [P(_Mask), P(_Grid), ctypes.c_int, ctypes.c_double,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                           ctypes.c_int64, ctypes.c_void_p,
+                                           ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.orc_tile_counts.restype = ctypes.c_int
+        lib.orc_tile_counts.argtypes = [P(_Mask), P(_Grid), ctypes.c_int64, ctypes.c_int,
+                                        ctypes.c_int, ctypes.c_int64, ctypes.c_void_p,
+                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
+        lib.orc_kept_pairs.restype = ctypes.c_int64
+        lib.orc_kept_pairs.argtypes = [P(_Mask), P(_Grid), ctypes.c_int]
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:  # pragma: no cover
+        return os.cpu_count() or 1
+
+
+def _mask(spec: Dict[str, int]) -> _Mask:
+    m = _Mask()
+    for k, _ in _Mask._fields_:
+        setattr(m, k, int(spec.get(k, 0)))
+    return m
+
+
+def _grid(grid: Sequence[int], unit: Sequence[int]) -> _Grid:
+    g = _Grid()
+    g.T, g.H, g.W = (int(x) for x in grid)
+    g.bt, g.bh, g.bw = (int(x) for x in unit)
+    return g
+
+
+def padded_tokens(grid, unit) -> int:
+    return int(_load().orc_padded_tokens(ctypes.byref(_grid(grid, unit))))
+
+
+def tile_major_order(grid, unit, n_slots: Optional[int] = None) -> np.ndarray:
+    """perm[slot] = natural token index or -1 (padding)."""
+    g = _grid(grid, unit)
+    if n_slots is None:
+        n_slots = padded_tokens(grid, unit)
+    perm = np.empty(n_slots, dtype=np.int32)
+    r = _load().orc_tile_major_order(ctypes.byref(g), n_slots, perm.ctypes.data)
+    if r < 0:
+        raise ValueError("n_slots smaller than the padded grid")
+    return perm
+
+
+def keep(spec, grid, unit, nq: int, nk: int) -> bool:
+    return bool(_load().orc_keep(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
+                                 int(nq), int(nk)))
+
+
+def keep_matrix(spec, grid, unit) -> np.ndarray:
+    N = int(np.prod(grid))
+    out = np.empty((N, N), dtype=np.uint8)
+    r = _load().orc_keep_matrix(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
+                                out.ctypes.data)
+    if r != 0:
+        raise ValueError("grid too large for a full predicate matrix")
+    return out.astype(bool)
+
+
+def attention_rows(spec, grid, unit, D: int, scale: float, q: np.ndarray, k: np.ndarray,
+                   v: np.ndarray, rows: Iterable[int], nthreads: Optional[int] = None
+                   ) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 masked attention for the given natural query rows of one (batch, head).
+
+    q, k, v: uint16 bf16 bits [N, D] in natural order.  Returns (o [R, D], lse [R]).
+    """
+    rows = np.ascontiguousarray(np.asarray(list(rows) if not isinstance(rows, np.ndarray)
+                                           else rows, dtype=np.int64))
+    q = np.ascontiguousarray(q, dtype=np.uint16)
+    k = np.ascontiguousarray(k, dtype=np.uint16)
+    v = np.ascontiguousarray(v, dtype=np.uint16)
+    N = int(np.prod(grid))
+    assert q.shape == (N, D) and k.shape == (N, D) and v.shape == (N, D)
+    o = np.zeros((len(rows), D), dtype=np.float64)
+    lse = np.zeros(len(rows), dtype=np.float64)
+    r = _load().orc_attention_rows(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
+                                   int(D), float(scale), q.ctypes.data, k.ctypes.data,
+                                   v.ctypes.data, len(rows), rows.ctypes.data,
+                                   o.ctypes.data, lse.ctypes.data,
+                                   int(nthreads or default_threads()))
+    if r != 0:
+        raise ValueError("bad arguments to orc_attention_rows")
+    return o, lse
+
+
+def tile_counts(spec, grid, unit, n_slots: int, Bq: int, Bk: int,
+                qtiles: Optional[Iterable[int]] = None, nthreads: Optional[int] = None
+                ) -> Tuple[np.ndarray, np.ndarray]:
+    """Brute-force kept-pair counts [len(qtiles), n_slots/Bk] and real queries per q tile."""
+    if qtiles is None:
+        qtiles = range(n_slots // Bq)
+    qt = np.ascontiguousarray(np.asarray(list(qtiles), dtype=np.int64))
+    counts = np.zeros((len(qt), n_slots // Bk), dtype=np.int64)
+    real_q = np.zeros(len(qt), dtype=np.int64)
+    r = _load().orc_tile_counts(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
+                                int(n_slots), int(Bq), int(Bk), len(qt), qt.ctypes.data,
+                                counts.ctypes.data, real_q.ctypes.data,
+                                int(nthreads or default_threads()))
+    if r != 0:
+        raise ValueError("bad arguments to orc_tile_counts")
+    return counts, real_q
+
+
+def classes_from_counts(counts: np.ndarray, real_q: np.ndarray, Bk: int) -> np.ndarray:
+    full = counts == (real_q[:, None] * Bk)
+    cls = np.where(counts == 0, 0, np.where(full, 2, 1)).astype(np.int8)
+    return cls
+
+
+def tile_map(spec, grid, unit, n_slots: int, Bq: int, Bk: int,
+             qtiles: Optional[Iterable[int]] = None, nthreads: Optional[int] = None
+             ) -> np.ndarray:
+    """int8 classes [len(qtiles), n_slots/Bk]: 0 empty, 1 boundary, 2 full."""
+    counts, real_q = tile_counts(spec, grid, unit, n_slots, Bq, Bk, qtiles, nthreads)
+    return classes_from_counts(counts, real_q, Bk)
+
+
+def kept_pairs(spec, grid, unit=(1, 1, 1), nthreads: Optional[int] = None) -> int:
+    return int(_load().orc_kept_pairs(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
+                                      int(nthreads or default_threads())))
