@@ -1,0 +1,112 @@
+// Token permutation between the natural (t,h,w) order and the tile-major
+// order of 3D units, with zero padding ("Video diffusion long-sequence
+// attention and sparsity", section 7.2: the permutation is one [N, d] gather;
+// "Parameterized Stripe Attention", key design 2: hierarchical layout with
+// 3D padding).  HBM-bound copies: every row of D bf16 values moves as 16-byte
+// vectors, a warp covers 2 rows (D = 128) or 4 rows (D = 64) per step, and
+// the grid is a multiple of the SM count with a grid-stride loop.
+#include <cuda_runtime.h>
+
+#include "vsa_internal.h"
+
+namespace {
+
+template <int D>
+__global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, long long rows,
+                                                      const uint4* __restrict__ in,
+                                                      uint4* __restrict__ out)
+{
+    constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
+    constexpr int RPW = 32 / VPR;     // rows per warp step
+    const int lane = threadIdx.x & 31;
+    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const int sub = lane / VPR, v = lane % VPR;
+    for (long long r = warp * RPW + sub; r < rows; r += nwarps * RPW) {
+        const long long bh = r / d.Nslots;
+        const long long p = r - bh * d.Nslots;
+        int t = 0, h = 0, w = 0;
+        uint4 val = make_uint4(0u, 0u, 0u, 0u);
+        if (vsa_slot_coords(d, p, t, h, w)) {
+            const long long n = ((long long)t * d.H + h) * d.W + w;
+            val = __ldg(in + (bh * d.N + n) * VPR + v);
+        }
+        out[r * VPR + v] = val;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, long long rows,
+                                                        const uint4* __restrict__ in,
+                                                        uint4* __restrict__ out)
+{
+    constexpr int VPR = D * 2 / 16;
+    constexpr int RPW = 32 / VPR;
+    const int lane = threadIdx.x & 31;
+    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const int sub = lane / VPR, v = lane % VPR;
+    const int HW = d.H * d.W;
+    for (long long r = warp * RPW + sub; r < rows; r += nwarps * RPW) {
+        const long long bh = r / d.N;
+        const long long n = r - bh * d.N;
+        const int t = (int)(n / HW);
+        const int rem = (int)(n - (long long)t * HW);
+        const int h = rem / d.W, w = rem - (rem / d.W) * d.W;
+        const long long p = vsa_token_slot(d, t, h, w);
+        out[r * VPR + v] = __ldg(in + (bh * d.Nslots + p) * VPR + v);
+    }
+}
+
+int sm_count()
+{
+    static int cached = 0;
+    if (!cached) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&cached, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            cached = 148;
+    }
+    return cached;
+}
+
+int launch(bool forward, vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream)
+{
+    if (!plan || B < 0) return VSA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+    if (B == 0) return VSA_OK;
+    if (!in || !out) return VSA_ERR_INVALID_ARG;
+    if (!vsa_aligned16(in) || !vsa_aligned16(out)) return VSA_ERR_ALIGNMENT;
+    const vsa_dims& d = plan->d;
+    const long long rows = (long long)B * d.heads * (forward ? d.Nslots : d.N);
+    const long long in_rows = (long long)B * d.heads * (forward ? d.N : d.Nslots);
+    const size_t row_bytes = (size_t)D * 2;
+    const char* ib = (const char*)in;
+    const char* ob = (const char*)out;
+    if (ib < ob + rows * row_bytes && ob < ib + in_rows * row_bytes) return VSA_ERR_INVALID_ARG;
+    const int threads = 256;
+    const long long want = (rows * (D * 2 / 16) + threads - 1) / threads;
+    const long long cap = (long long)sm_count() * 8;
+    const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (forward) {
+        if (D == 128) permute_kernel<128><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+        else permute_kernel<64><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+    } else {
+        if (D == 128) unpermute_kernel<128><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+        else unpermute_kernel<64><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+    }
+    return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int vsa_permute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream)
+{
+    return launch(true, plan, in, out, B, D, stream);
+}
+
+extern "C" int vsa_unpermute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream)
+{
+    return launch(false, plan, in, out, B, D, stream);
+}

@@ -1,0 +1,601 @@
+// Plan construction: mask specs -> tile map, per-query-block kv-tile lists,
+// kv-tile segment table and stripe offset tables, all built by GPU kernels.
+//
+// Tile classes follow the three kinds of "Sparse VideoGen: accelerating video
+// diffusion attention on TPU" (section "logical sparsity is not physical
+// sparsity"); the per-query-block list of kv tiles is the block-sparse
+// interface of "Video diffusion long-sequence attention and sparsity",
+// section 7.3.
+//
+// Classification is exact without visiting element pairs: the real tokens of
+// a tile form one or a few 3D boxes (a tile is a box inside one unit or a run
+// of whole units), and every mask is (relation on t) AND (relation on the
+// in-frame position), OR the frame-0 sink.  For a pair of boxes the kept set
+// is therefore the product of a t-pair set and an (h,w)-pair set, so "some
+// pair kept" and "every pair kept" follow from per-axis any/all tests.  The
+// in-frame stripe relation depends on s_k - s_q only, so for each pair of
+// latent rows the kept pairs are the offsets of a contiguous range, read
+// from a per-head bit table over all offsets.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+
+#include "vsa_internal.h"
+
+namespace {
+
+struct Box {
+    int t0, t1, h0, h1, w0, w1;  // half-open real ranges
+};
+
+// Box i of tile `tile` (size B slots).  Returns false when that box holds no
+// real token.  Sets *pad when the tile holds any padding slot.
+__device__ bool tile_box(const vsa_dims& d, int tile, int B, int i, Box& bx, bool& pad)
+{
+    const long long p0 = (long long)tile * B;
+    int u, t0, t1, h0, h1, w0, w1;
+    if (B <= d.U) {
+        if (p0 >= d.Npad) { pad = true; return false; }
+        u = (int)(p0 / d.U);
+        const int o0 = (int)(p0 - (long long)u * d.U);
+        const int per_t = d.nTh * d.nTw;
+        const int tt = u / per_t, th = (u - tt * per_t) / d.nTw, tw = u - tt * per_t - th * d.nTw;
+        const int hw = d.bh * d.bw;
+        const int ot = o0 / hw, oh = (o0 - ot * hw) / d.bw, ow = o0 - ot * hw - oh * d.bw;
+        if (B % hw == 0) {
+            t0 = tt * d.bt + ot; t1 = t0 + B / hw;
+            h0 = th * d.bh; h1 = h0 + d.bh;
+            w0 = tw * d.bw; w1 = w0 + d.bw;
+        } else if (B % d.bw == 0) {
+            t0 = tt * d.bt + ot; t1 = t0 + 1;
+            h0 = th * d.bh + oh; h1 = h0 + B / d.bw;
+            w0 = tw * d.bw; w1 = w0 + d.bw;
+        } else {
+            t0 = tt * d.bt + ot; t1 = t0 + 1;
+            h0 = th * d.bh + oh; h1 = h0 + 1;
+            w0 = tw * d.bw + ow; w1 = w0 + B;
+        }
+    } else {
+        u = (int)(p0 / d.U) + i;
+        if ((long long)u * d.U >= d.Npad) { pad = true; return false; }
+        const int per_t = d.nTh * d.nTw;
+        const int tt = u / per_t, th = (u - tt * per_t) / d.nTw, tw = u - tt * per_t - th * d.nTw;
+        t0 = tt * d.bt; t1 = t0 + d.bt;
+        h0 = th * d.bh; h1 = h0 + d.bh;
+        w0 = tw * d.bw; w1 = w0 + d.bw;
+    }
+    if (t1 > d.T || h1 > d.H || w1 > d.W) pad = true;
+    bx.t0 = t0; bx.t1 = min(t1, d.T);
+    bx.h0 = h0; bx.h1 = min(h1, d.H);
+    bx.w0 = w0; bx.w1 = min(w1, d.W);
+    return bx.t0 < bx.t1 && bx.h0 < bx.h1 && bx.w0 < bx.w1;
+}
+
+__device__ __forceinline__ bool rel_t(const vsa_mask_spec& m, const vsa_dims& d, int tq, int tk)
+{
+    switch (m.kind) {
+    case VSA_MASK_SVG_SPATIAL: return vsa_iabs(tk - tq) <= m.rt;
+    case VSA_MASK_STRIPE: return (vsa_iabs(tk - tq - m.To) % m.Ts) <= m.Tw - 1;
+    case VSA_MASK_STA: {
+        const int s = vsa_sta_start(tq / d.bt, d.nTt, m.kt);
+        const int uk = tk / d.bt;
+        return uk >= s && uk < s + min(m.kt, d.nTt);
+    }
+    default: return true;
+    }
+}
+
+// Interval helpers for |a - b| over a in [a0,a1), b in [b0,b1).
+__device__ __forceinline__ int min_absdiff(int a0, int a1, int b0, int b1)
+{
+    if (b0 > a1 - 1) return b0 - (a1 - 1);
+    if (a0 > b1 - 1) return a0 - (b1 - 1);
+    return 0;
+}
+__device__ __forceinline__ int max_absdiff(int a0, int a1, int b0, int b1)
+{
+    return max(b1 - 1 - a0, a1 - 1 - b0);
+}
+
+// Number of set bits of `tab` in bit positions [i0, i1] (inclusive).
+__device__ __forceinline__ int count_bits(const uint32_t* tab, int i0, int i1)
+{
+    int c = 0;
+    const int wa = i0 >> 5, wb = i1 >> 5;
+    for (int wd = wa; wd <= wb; ++wd) {
+        uint32_t m = tab[wd];
+        const int lo = (wd == wa) ? (i0 & 31) : 0;
+        const int hi = (wd == wb) ? (i1 & 31) : 31;
+        m &= (0xFFFFFFFFu >> (31 - hi)) & (0xFFFFFFFFu << lo);
+        c += __popc(m);
+    }
+    return c;
+}
+
+// any / all of the in-frame relation over (A.h x A.w) x (B.h x B.w).
+__device__ void rel_s(const vsa_mask_spec& m, const vsa_dims& d, const uint32_t* sbits,
+                      const Box& A, const Box& B, bool& any, bool& all)
+{
+    switch (m.kind) {
+    case VSA_MASK_SVG_TEMPORAL: {
+        const bool anyh = min_absdiff(A.h0, A.h1, B.h0, B.h1) <= m.rh;
+        const bool allh = max_absdiff(A.h0, A.h1, B.h0, B.h1) <= m.rh;
+        const bool anyw = min_absdiff(A.w0, A.w1, B.w0, B.w1) <= m.rw;
+        const bool allw = max_absdiff(A.w0, A.w1, B.w0, B.w1) <= m.rw;
+        any = anyh && anyw;
+        all = allh && allw;
+        return;
+    }
+    case VSA_MASK_STA: {
+        const int sh = vsa_sta_start(A.h0 / d.bh, d.nTh, m.kh), uh = B.h0 / d.bh;
+        const int sw = vsa_sta_start(A.w0 / d.bw, d.nTw, m.kw), uw = B.w0 / d.bw;
+        const bool in = uh >= sh && uh < sh + min(m.kh, d.nTh) && uw >= sw && uw < sw + min(m.kw, d.nTw);
+        any = in;
+        all = in;
+        return;
+    }
+    case VSA_MASK_STRIPE: {
+        const int HW1 = d.H * d.W - 1;
+        const int dlo = B.w0 - (A.w1 - 1), dhi = (B.w1 - 1) - A.w0;
+        any = false;
+        all = true;
+        for (int hq = A.h0; hq < A.h1; ++hq) {
+            for (int hk = B.h0; hk < B.h1; ++hk) {
+                const int x0 = (hk - hq) * d.W + dlo + HW1, x1 = (hk - hq) * d.W + dhi + HW1;
+                const int ones = count_bits(sbits, x0, x1);
+                any = any || ones > 0;
+                all = all && ones == x1 - x0 + 1;
+                if (any && !all) return;
+            }
+        }
+        return;
+    }
+    default:
+        any = true;
+        all = true;
+        return;
+    }
+}
+
+// any / all kept over real (A x B).
+__device__ void classify_boxes(const vsa_mask_spec& m, const vsa_dims& d, const uint32_t* sbits,
+                               const Box& A, const Box& B, bool& any, bool& all)
+{
+    const bool sinkk = m.sink && B.t0 == 0;
+    const int tk0 = sinkk ? 1 : B.t0;
+    if (tk0 >= B.t1) {  // the key box is frame 0 only and every pair is kept by the sink
+        any = true;
+        all = true;
+        return;
+    }
+    bool anyt = false, allt = true;
+    for (int tq = A.t0; tq < A.t1; ++tq)
+        for (int tk = tk0; tk < B.t1; ++tk) {
+            const bool r = rel_t(m, d, tq, tk);
+            anyt = anyt || r;
+            allt = allt && r;
+        }
+    bool anys = false, alls = false;
+    if (anyt || allt) rel_s(m, d, sbits, A, B, anys, alls);
+    any = sinkk || (anyt && anys);
+    all = allt && alls;
+}
+
+__global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                const uint32_t* __restrict__ sbits, int8_t* __restrict__ map)
+{
+    const long long per_head = (long long)d.nQ * d.nK;
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= per_head * d.heads) return;
+    const int head = (int)(idx / per_head);
+    const long long rem = idx - (long long)head * per_head;
+    const int a = (int)(rem / d.nK), b = (int)(rem - (long long)a * d.nK);
+    const vsa_mask_spec m = specs[head];
+    const uint32_t* sb = sbits ? sbits + (size_t)head * d.sbits_words : nullptr;
+    const int nqb = d.Bq <= d.U ? 1 : d.Bq / d.U;
+    const int nkb = d.Bk <= d.U ? 1 : d.Bk / d.U;
+
+    bool qpad = false, kpad = false, anyq = false;
+    bool any = false, all = true;
+    for (int i = 0; i < nqb && !(any && !all); ++i) {
+        Box A;
+        if (!tile_box(d, a, d.Bq, i, A, qpad)) continue;
+        anyq = true;
+        for (int j = 0; j < nkb; ++j) {
+            Box B;
+            if (!tile_box(d, b, d.Bk, j, B, kpad)) continue;
+            bool ba, bl;
+            classify_boxes(m, d, sb, A, B, ba, bl);
+            any = any || ba;
+            all = all && bl;
+            if (any && !all) break;
+        }
+    }
+    // padding anywhere in the kv tile rules out "full"
+    if (!kpad) {
+        for (int j = 0; j < nkb; ++j) {
+            Box B;
+            if (!tile_box(d, b, d.Bk, j, B, kpad)) kpad = true;
+        }
+    }
+    int8_t cls = VSA_TILE_EMPTY;
+    if (anyq && any) cls = (all && !kpad) ? VSA_TILE_FULL : VSA_TILE_BOUNDARY;
+    map[idx] = cls;
+}
+
+// Per kv tile, one entry per run of bw slots sharing (t, h): the run's t, h,
+// first w and number of real tokens.
+__global__ void seg_table_kernel(vsa_dims d, int2* __restrict__ seg)
+{
+    const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (long long)d.nK * d.nseg) return;
+    const long long p = idx * d.bw;  // first slot of the run
+    int t = 0, h = 0, w0 = 0, nv = 0;
+    if (p < d.Npad) {
+        int w;
+        vsa_slot_coords(d, p, t, h, w);
+        w0 = w;
+        if (t < d.T && h < d.H) nv = max(0, min(d.bw, d.W - w0));
+    }
+    seg[idx] = make_int2((t & 0xFFFF) | (h << 16), (w0 & 0xFFFF) | (nv << 16));
+}
+
+// Stripe in-frame relation over every offset x = s_k - s_q in [-(HW-1), HW-1]:
+// bit (x + HW - 1) = ((|x - So| mod Ss) <= Sw - 1).
+__global__ void stripe_bits_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                   uint32_t* __restrict__ sbits)
+{
+    const int head = blockIdx.y;
+    const int wd = blockIdx.x * blockDim.x + threadIdx.x;
+    if (wd >= d.sbits_words) return;
+    const vsa_mask_spec m = specs[head];
+    uint32_t v = 0;
+    if (m.kind == VSA_MASK_STRIPE) {
+        const int HW = d.H * d.W;
+        for (int i = 0; i < 32; ++i) {
+            const int x = wd * 32 + i - (HW - 1);
+            if (x > HW - 1) break;
+            if ((vsa_iabs(x - m.So) % m.Ss) <= m.Sw - 1) v |= 1u << i;
+        }
+    }
+    sbits[(size_t)head * d.sbits_words + wd] = v;
+}
+
+// One warp per (head, execution block): the ordered list of kv tiles with a
+// kept pair for either 64-row half, with both halves' classes, plus tile and
+// step totals.
+__global__ void kv_list_kernel(vsa_dims d, const int8_t* __restrict__ map,
+                               int32_t* __restrict__ list_cnt, int32_t* __restrict__ list,
+                               unsigned long long* __restrict__ counts,
+                               unsigned long long* __restrict__ steps)
+{
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)d.heads * d.nE) return;
+    const int head = (int)(gw / d.nE), e = (int)(gw - (long long)head * d.nE);
+    int r0, r1;
+    bool own0, own1;
+    if (d.Bq == 64) { r0 = 2 * e; r1 = 2 * e + 1; own0 = true; own1 = true; }
+    else if (d.Bq == 128) { r0 = e; r1 = e; own0 = true; own1 = false; }
+    else { r0 = e >> 1; r1 = r0; own0 = (e & 1) == 0; own1 = false; }
+    const int8_t* m0 = map + ((size_t)head * d.nQ + r0) * d.nK;
+    const int8_t* m1 = map + ((size_t)head * d.nQ + r1) * d.nK;
+    int32_t* out = list + ((size_t)head * d.nE + e) * d.nK;
+    int cnt = 0;
+    unsigned c[3] = {0, 0, 0};
+    for (int jb = 0; jb < d.nK; jb += 32) {
+        const int j = jb + lane;
+        int c0 = 0, c1 = 0;
+        if (j < d.nK) {
+            c0 = m0[j];
+            c1 = m1[j];
+            if (own0) c[c0] += 1;
+            if (own1) c[c1] += 1;
+        }
+        const bool nz = (c0 | c1) != 0;
+        const unsigned bal = __ballot_sync(0xFFFFFFFFu, nz);
+        if (nz) {
+            const int pos = cnt + __popc(bal & ((1u << lane) - 1u));
+            out[pos] = j | (c0 << 24) | (c1 << 26);
+        }
+        cnt += __popc(bal);
+    }
+    for (int k = 0; k < 3; ++k)
+        for (int off = 16; off > 0; off >>= 1) c[k] += __shfl_xor_sync(0xFFFFFFFFu, c[k], off);
+    if (lane == 0) {
+        list_cnt[(size_t)head * d.nE + e] = cnt;
+        atomicAdd(&steps[head], (unsigned long long)cnt);
+        for (int k = 0; k < 3; ++k)
+            if (c[k]) atomicAdd(&counts[head * 3 + k], (unsigned long long)c[k]);
+    }
+}
+
+__global__ void perm_kernel(vsa_dims d, int32_t* __restrict__ perm)
+{
+    const long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= d.Nslots) return;
+    int t, h, w;
+    perm[p] = vsa_slot_coords(d, p, t, h, w) ? (int32_t)(((long long)t * d.H + h) * d.W + w) : -1;
+}
+
+bool tile_fits_unit(int B, int U, int bh, int bw)
+{
+    if (B >= U) return B % U == 0;
+    if (U % B) return false;
+    const int hw = bh * bw;
+    return (B % hw == 0) || (B % bw == 0 && hw % B == 0) || (bw % B == 0);
+}
+
+unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
+
+}  // namespace
+
+int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
+{
+    const vsa_dims& d = p->d;
+    VSA_CUDA_TRY(cudaMemsetAsync(p->d_counts, 0, sizeof(unsigned long long) * 3 * d.heads, s));
+    VSA_CUDA_TRY(cudaMemsetAsync(p->d_steps, 0, sizeof(unsigned long long) * d.heads, s));
+    seg_table_kernel<<<blocks_for((long long)d.nK * d.nseg, 256), 256, 0, s>>>(d, p->d_seg);
+    VSA_CUDA_TRY(cudaGetLastError());
+    if (p->has_stripe) {
+        dim3 g(blocks_for(d.sbits_words, 128), d.heads);
+        stripe_bits_kernel<<<g, 128, 0, s>>>(d, p->d_specs, p->d_sbits);
+        VSA_CUDA_TRY(cudaGetLastError());
+    }
+    const long long cells = (long long)d.heads * d.nQ * d.nK;
+    tile_map_kernel<<<blocks_for(cells, 256), 256, 0, s>>>(d, p->d_specs,
+                                                          p->has_stripe ? p->d_sbits : nullptr,
+                                                          p->d_map);
+    VSA_CUDA_TRY(cudaGetLastError());
+    kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
+        d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
+    VSA_CUDA_TRY(cudaGetLastError());
+    return VSA_OK;
+}
+
+static int validate_spec(const vsa_mask_spec& m)
+{
+    if (m.kind < VSA_MASK_FULL || m.kind > VSA_MASK_STRIPE) return VSA_ERR_INVALID_ARG;
+    if (m.sink != 0 && m.sink != 1) return VSA_ERR_INVALID_ARG;
+    const int lim = 1 << 20;
+    switch (m.kind) {
+    case VSA_MASK_SVG_SPATIAL:
+        if (m.rt < 0 || m.rt > lim) return VSA_ERR_INVALID_ARG;
+        break;
+    case VSA_MASK_SVG_TEMPORAL:
+        if (m.rh < 0 || m.rw < 0 || m.rh > lim || m.rw > lim) return VSA_ERR_INVALID_ARG;
+        break;
+    case VSA_MASK_STA:
+        if (m.kt < 1 || m.kh < 1 || m.kw < 1) return VSA_ERR_INVALID_ARG;
+        break;
+    case VSA_MASK_STRIPE:
+        if (m.Tw < 1 || m.Ts < 1 || m.Sw < 1 || m.Ss < 1) return VSA_ERR_INVALID_ARG;
+        if (m.To < -lim || m.To > lim || m.So < -lim || m.So > lim || m.Tw > lim || m.Sw > lim ||
+            m.Ts > lim || m.Ss > lim)
+            return VSA_ERR_INVALID_ARG;
+        break;
+    default:
+        break;
+    }
+    return VSA_OK;
+}
+
+static void free_plan(vsa_plan_s* p)
+{
+    if (!p) return;
+    cudaFree(p->d_specs);
+    cudaFree(p->d_map);
+    cudaFree(p->d_list_cnt);
+    cudaFree(p->d_list);
+    cudaFree(p->d_seg);
+    cudaFree(p->d_sbits);
+    cudaFree(p->d_counts);
+    cudaFree(p->d_steps);
+    cudaFree(p->d_status);
+    delete p;
+}
+
+// Validates the grid / unit / tile arguments and derives every shape of a plan.
+static int compute_dims(int num_heads, int T, int H, int W, int bt, int bh, int bw, int q_tile,
+                        int kv_tile, int has_stripe, vsa_dims* out)
+{
+    if (num_heads < 1 || T < 1 || H < 1 || W < 1 || bt < 1 || bh < 1 || bw < 1)
+        return VSA_ERR_INVALID_ARG;
+    if (T > 32767 || H > 32767 || W > 32767 || bt > 32767 || bh > 32767) return VSA_ERR_UNSUPPORTED;
+    if (q_tile != 64 && q_tile != 128 && q_tile != 256) return VSA_ERR_UNSUPPORTED;
+    if (kv_tile != 64 && kv_tile != 128) return VSA_ERR_UNSUPPORTED;
+    if (bw > 32 || (bw & (bw - 1))) return VSA_ERR_UNSUPPORTED;
+    vsa_dims d;
+    memset(&d, 0, sizeof d);
+    d.T = T; d.H = H; d.W = W; d.bt = bt; d.bh = bh; d.bw = bw;
+    d.Tp = (T + bt - 1) / bt * bt;
+    d.Hp = (H + bh - 1) / bh * bh;
+    d.Wp = (W + bw - 1) / bw * bw;
+    if (d.Tp > 32767 || d.Hp > 32767 || d.Wp > 32767) return VSA_ERR_UNSUPPORTED;
+    d.nTt = d.Tp / bt; d.nTh = d.Hp / bh; d.nTw = d.Wp / bw;
+    const long long U = (long long)bt * bh * bw;
+    if (U > (1 << 24)) return VSA_ERR_UNSUPPORTED;
+    d.U = (int)U;
+    if (!tile_fits_unit(q_tile, d.U, bh, bw) || !tile_fits_unit(kv_tile, d.U, bh, bw))
+        return VSA_ERR_UNSUPPORTED;
+    if (has_stripe && (long long)H * W > 65536) return VSA_ERR_UNSUPPORTED;
+    d.heads = num_heads;
+    d.Bq = q_tile; d.Bk = kv_tile;
+    d.N = (long long)T * H * W;
+    d.Npad = (long long)d.Tp * d.Hp * d.Wp;
+    const long long L = std::max(VSA_EXEC_ROWS, std::max(q_tile, kv_tile));
+    d.Nslots = (d.Npad + L - 1) / L * L;
+    if (d.Nslots > (1LL << 24)) return VSA_ERR_UNSUPPORTED;  // 24-bit kv tile index, int32 rows
+    d.nQ = (int)(d.Nslots / q_tile);
+    d.nK = (int)(d.Nslots / kv_tile);
+    d.nE = (int)(d.Nslots / VSA_EXEC_ROWS);
+    d.nseg = kv_tile / bw;
+    d.sbits_words = has_stripe ? (int)((2LL * H * W - 1 + 31) / 32 + 1) : 0;
+    *out = d;
+    return VSA_OK;
+}
+
+static void fill_info(const vsa_dims& d, vsa_plan_info_t* out)
+{
+    out->T = d.T; out->H = d.H; out->W = d.W;
+    out->bt = d.bt; out->bh = d.bh; out->bw = d.bw;
+    out->num_heads = d.heads;
+    out->q_tile = d.Bq; out->kv_tile = d.Bk;
+    out->n_q_tiles = d.nQ; out->n_kv_tiles = d.nK;
+    out->n_tokens = d.N; out->n_padded = d.Npad; out->n_slots = d.Nslots;
+    out->map_bytes = (int64_t)d.heads * d.nQ * d.nK;
+}
+
+extern "C" int vsa_layout_info(int num_heads, int T, int H, int W, int bt, int bh, int bw, int q_tile,
+                               int kv_tile, vsa_plan_info_t* out)
+{
+    if (!out) return VSA_ERR_INVALID_ARG;
+    vsa_dims d;
+    const int r = compute_dims(num_heads, T, H, W, bt, bh, bw, q_tile, kv_tile, 0, &d);
+    if (r != VSA_OK) return r;
+    fill_info(d, out);
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T, int H, int W,
+                               int bt, int bh, int bw, int q_tile, int kv_tile, void* stream,
+                               vsa_plan_t* out)
+{
+    if (!out) return VSA_ERR_INVALID_ARG;
+    *out = nullptr;
+    if (!specs || num_heads < 1) return VSA_ERR_INVALID_ARG;
+    int has_stripe = 0;
+    for (int h = 0; h < num_heads; ++h) {
+        const int r = validate_spec(specs[h]);
+        if (r != VSA_OK) return r;
+        has_stripe |= specs[h].kind == VSA_MASK_STRIPE;
+    }
+    vsa_dims d;
+    {
+        const int r = compute_dims(num_heads, T, H, W, bt, bh, bw, q_tile, kv_tile, has_stripe, &d);
+        if (r != VSA_OK) return r;
+    }
+
+    vsa_plan_s* p = new (std::nothrow) vsa_plan_s;
+    if (!p) return VSA_ERR_OOM;
+    memset(p, 0, sizeof *p);
+    p->d = d;
+    p->has_stripe = has_stripe;
+    if (cudaGetDevice(&p->device) != cudaSuccess) { delete p; return VSA_ERR_CUDA; }
+    bool ok = true;
+    ok = ok && cudaMalloc(&p->d_specs, sizeof(vsa_mask_spec) * num_heads) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_map, (size_t)num_heads * d.nQ * d.nK) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_list_cnt, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_list, sizeof(int32_t) * (size_t)num_heads * d.nE * d.nK) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_seg, sizeof(int2) * (size_t)d.nK * d.nseg) == cudaSuccess;
+    if (has_stripe)
+        ok = ok && cudaMalloc(&p->d_sbits, sizeof(uint32_t) * (size_t)num_heads * d.sbits_words) ==
+                       cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_counts, sizeof(unsigned long long) * 3 * num_heads) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_steps, sizeof(unsigned long long) * num_heads) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_status, sizeof(unsigned int)) == cudaSuccess;
+    if (!ok) {
+        cudaGetLastError();
+        free_plan(p);
+        return VSA_ERR_OOM;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaMemcpyAsync(p->d_specs, specs, sizeof(vsa_mask_spec) * num_heads, cudaMemcpyHostToDevice,
+                        s) != cudaSuccess ||
+        cudaMemsetAsync(p->d_status, 0, sizeof(unsigned int), s) != cudaSuccess) {
+        free_plan(p);
+        return VSA_ERR_CUDA;
+    }
+    // the host copy of specs may be released as soon as the copy is done
+    if (cudaStreamSynchronize(s) != cudaSuccess) {
+        free_plan(p);
+        return VSA_ERR_CUDA;
+    }
+    const int r = vsa_build_plan_kernels(p, s);
+    if (r != VSA_OK) {
+        free_plan(p);
+        return r;
+    }
+    *out = p;
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_build(vsa_plan_t plan, void* stream)
+{
+    if (!plan) return VSA_ERR_INVALID_ARG;
+    return vsa_build_plan_kernels(plan, (cudaStream_t)stream);
+}
+
+extern "C" int vsa_plan_info(vsa_plan_t plan, vsa_plan_info_t* out)
+{
+    if (!plan || !out) return VSA_ERR_INVALID_ARG;
+    fill_info(plan->d, out);
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_tile_map(vsa_plan_t plan, int8_t* host_dst, size_t bytes, void* stream)
+{
+    if (!plan || !host_dst) return VSA_ERR_INVALID_ARG;
+    const size_t need = (size_t)plan->d.heads * plan->d.nQ * plan->d.nK;
+    if (bytes < need) return VSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    VSA_CUDA_TRY(cudaMemcpyAsync(host_dst, plan->d_map, need, cudaMemcpyDeviceToHost, s));
+    VSA_CUDA_TRY(cudaStreamSynchronize(s));
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_tile_counts(vsa_plan_t plan, int64_t* host_counts, size_t n, void* stream)
+{
+    if (!plan || !host_counts || n < (size_t)3 * plan->d.heads) return VSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    VSA_CUDA_TRY(cudaMemcpyAsync(host_counts, plan->d_counts,
+                                 sizeof(unsigned long long) * 3 * plan->d.heads,
+                                 cudaMemcpyDeviceToHost, s));
+    VSA_CUDA_TRY(cudaStreamSynchronize(s));
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream)
+{
+    if (!plan || !host_dst || n < (size_t)plan->d.heads) return VSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    VSA_CUDA_TRY(cudaMemcpyAsync(host_dst, plan->d_steps, sizeof(unsigned long long) * plan->d.heads,
+                                 cudaMemcpyDeviceToHost, s));
+    VSA_CUDA_TRY(cudaStreamSynchronize(s));
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream)
+{
+    if (!plan || !host_dst || n < (size_t)plan->d.Nslots) return VSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    int32_t* tmp = nullptr;
+    if (cudaMalloc(&tmp, sizeof(int32_t) * plan->d.Nslots) != cudaSuccess) {
+        cudaGetLastError();
+        return VSA_ERR_OOM;
+    }
+    perm_kernel<<<blocks_for(plan->d.Nslots, 256), 256, 0, s>>>(plan->d, tmp);
+    cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(host_dst, tmp, sizeof(int32_t) * plan->d.Nslots, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(tmp);
+    return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+extern "C" int vsa_plan_destroy(vsa_plan_t plan)
+{
+    if (!plan) return VSA_ERR_INVALID_ARG;
+    int prev = -1;
+    const int dev = plan->device;
+    cudaGetDevice(&prev);
+    if (prev != dev) cudaSetDevice(dev);
+    const cudaError_t e = cudaDeviceSynchronize();
+    free_plan(plan);
+    if (prev >= 0 && prev != dev) cudaSetDevice(prev);
+    return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}

@@ -1,0 +1,202 @@
+/*
+ * vsa -- block-sparse attention over a flattened 3D video token grid, for B200
+ * (sm_100a).  C ABI: plain pointers, sizes and status codes; no C++ types, no
+ * exceptions cross it.
+ *
+ * Call order for one attention layer:
+ *
+ *   vsa_plan_create   mask specs + grid + 3D unit + tile shape
+ *                     -> int8 tile map, per-query-block kv-tile lists,
+ *                        tile-major token order (built on the GPU)
+ *   vsa_permute       q, k, v  natural [B,Hh,N,D] -> tile-major [B,Hh,n_slots,D]
+ *   vsa_sparse_attn_fwd       tile-major q,k,v -> tile-major o, lse
+ *   vsa_unpermute     o  tile-major -> natural [B,Hh,N,D]
+ *
+ * Sources (web pages on block-sparse video attention):
+ *  [SVG-TPU] "Sparse VideoGen: accelerating video diffusion attention on TPU"
+ *  [PSA]     "Parameterized Stripe Attention for Efficient Video Generation"
+ *  [STA]     "Fast Video Generation with Sliding Tile Attention" (explainer)
+ *  [VDS]     "Video diffusion long-sequence attention and sparsity", section 7
+ *
+ * Token order.  The natural order flattens (t,h,w) with t slowest:
+ * n = (t*H + h)*W + w ([VDS] section 7.2).  The tile-major order pads each
+ * axis to a multiple of the 3D unit (bt,bh,bw) (T' = ceil(T/bt)*bt, [PSA] key
+ * design 2), lists units in (t,h,w) row-major order and, inside a unit, tokens
+ * in (t,h,w) row-major order, so the tokens of a unit are contiguous ([STA]
+ * section 3).  The slot count n_slots is the padded token count rounded up to
+ * a multiple of max(128, q_tile, kv_tile); every slot that holds no real token
+ * is padding.  Padding keys never receive attention weight ([SVG-TPU],
+ * "aligning the sparse mask with execution").
+ *
+ * Memory.  The caller owns q, k, v, o and lse (device memory, contiguous,
+ * 16-byte aligned).  A plan owns its device buffers and is immutable after
+ * creation; vsa_plan_build may rewrite them in place.  vsa_permute,
+ * vsa_unpermute and vsa_sparse_attn_fwd allocate nothing.
+ *
+ * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  Every launch is asynchronous on that stream; host-visible results
+ * (tile maps, counts, status) are read by the calls documented as synchronous.
+ *
+ * Errors.  Every call returns VSA_OK (0) or a negative code.  Argument errors
+ * are detected on the host before any launch.  A device-side watchdog turns a
+ * wait that cannot complete into VSA_ERR_TIMEOUT, reported by
+ * vsa_check_status; no kernel traps or spins without bound.
+ */
+#ifndef VSA_H
+#define VSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VSA_VERSION 1
+
+enum {
+    VSA_OK = 0,
+    VSA_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad enum      */
+    VSA_ERR_UNSUPPORTED = -2, /* valid but not implemented: D, tile/unit shape  */
+    VSA_ERR_ALIGNMENT = -3,   /* a tensor pointer is not 16-byte aligned        */
+    VSA_ERR_CUDA = -4,        /* a CUDA runtime / driver call failed            */
+    VSA_ERR_OOM = -5,         /* device allocation failed (vsa_plan_create)     */
+    VSA_ERR_TIMEOUT = -6,     /* a kernel's bounded wait expired (watchdog)     */
+    VSA_ERR_DEVICE = -7       /* a kernel flagged an inconsistent state         */
+};
+
+/* Mask families.
+ *  FULL          keep every real key.
+ *  SVG_SPATIAL   keep iff |t_k - t_q| <= rt                     ([SVG-TPU] SVG heads)
+ *  SVG_TEMPORAL  keep iff |h_k - h_q| <= rh and |w_k - w_q| <= rw ([SVG-TPU] SVG heads)
+ *  STA           keep iff the key's 3D unit lies in the query unit's window of
+ *                kt x kh x kw units; the window is centred on the query's unit
+ *                and shifted inward at the grid edge so that it always holds
+ *                min(k, units on that axis) units ([STA] section 3, Eq. 4)
+ *  STRIPE        keep iff (|t_k - t_q - To| mod Ts) <= Tw - 1 and
+ *                (|s_k - s_q - So| mod Ss) <= Sw - 1, s = h*W + w ([PSA] key design 1)
+ * With sink = 1 every query also keeps every real key of frame 0 (t_k = 0),
+ * the attention sink both SVG masks keep ([SVG-TPU] figure 3).  All
+ * coordinates are real (unpadded) grid coordinates. */
+typedef enum {
+    VSA_MASK_FULL = 0,
+    VSA_MASK_SVG_SPATIAL = 1,
+    VSA_MASK_SVG_TEMPORAL = 2,
+    VSA_MASK_STA = 3,
+    VSA_MASK_STRIPE = 4
+} vsa_mask_kind;
+
+typedef struct {
+    int32_t kind;            /* vsa_mask_kind                                    */
+    int32_t sink;            /* 0 or 1                                           */
+    int32_t rt, rh, rw;      /* SVG radii (>= 0)                                 */
+    int32_t kt, kh, kw;      /* STA window in units (>= 1)                       */
+    int32_t Tw, To, Ts;      /* stripe, inter-frame: width >= 1, offset, stride >= 1 */
+    int32_t Sw, So, Ss;      /* stripe, intra-frame: width >= 1, offset, stride >= 1 */
+} vsa_mask_spec;
+
+typedef struct vsa_plan_s* vsa_plan_t;
+
+typedef struct {
+    int32_t T, H, W;          /* real latent grid                                */
+    int32_t bt, bh, bw;       /* 3D unit                                         */
+    int32_t num_heads;
+    int32_t q_tile, kv_tile;  /* tile-map granularity (rows of q / k per tile)   */
+    int32_t n_q_tiles, n_kv_tiles;
+    int64_t n_tokens;         /* T*H*W                                           */
+    int64_t n_padded;         /* T'H'W'                                          */
+    int64_t n_slots;          /* rows of every tile-major tensor                 */
+    int64_t map_bytes;        /* num_heads * n_q_tiles * n_kv_tiles              */
+} vsa_plan_info_t;
+
+/* Tile classes stored in the map ([SVG-TPU], "logical sparsity is not
+ * physical sparsity"): a (q tile, kv tile) pair is EMPTY when no (real query,
+ * key slot) pair is kept, FULL when every such pair is kept (so a kv tile that
+ * holds padding is never full), BOUNDARY otherwise. */
+enum { VSA_TILE_EMPTY = 0, VSA_TILE_BOUNDARY = 1, VSA_TILE_FULL = 2 };
+
+/* Build a plan for `num_heads` heads (specs[h] for head h) on the T x H x W
+ * grid with 3D unit (bt,bh,bw) and tile shape q_tile x kv_tile.
+ * Supported: q_tile in {64,128,256}, kv_tile in {64,128}; bw in
+ * {1,2,4,8,16,32} dividing kv_tile; each tile either a whole number of units
+ * or one box inside a unit (its size a multiple of bh*bw, or of bw and
+ * dividing bh*bw, or dividing bw); T, H, W < 32768; H*W <= 65536 for stripe heads.
+ * Allocates the plan's device buffers on the current device and launches the
+ * build kernels on `stream` (asynchronous).  On error *out is left NULL. */
+int vsa_plan_create(const vsa_mask_spec* specs, int num_heads,
+                    int T, int H, int W, int bt, int bh, int bw,
+                    int q_tile, int kv_tile, void* stream, vsa_plan_t* out);
+
+/* Host-only: the shapes a plan with these arguments would have (n_slots,
+ * tile counts, map size), for sizing buffers before vsa_plan_create.  Same
+ * argument checks as vsa_plan_create (stripe heads are not considered). */
+int vsa_layout_info(int num_heads, int T, int H, int W, int bt, int bh, int bw,
+                    int q_tile, int kv_tile, vsa_plan_info_t* out);
+
+/* Re-run the build kernels (tile map, kv-tile lists, tables) into the plan's
+ * own buffers.  Asynchronous, allocates nothing. */
+int vsa_plan_build(vsa_plan_t plan, void* stream);
+
+/* Host-side shape information; no device work. */
+int vsa_plan_info(vsa_plan_t plan, vsa_plan_info_t* out);
+
+/* Synchronous: copies the int8 map [num_heads][n_q_tiles][n_kv_tiles] to host
+ * memory `host_dst` of `bytes` >= map_bytes. */
+int vsa_plan_tile_map(vsa_plan_t plan, int8_t* host_dst, size_t bytes, void* stream);
+
+/* Synchronous: per-head tile totals, host_counts[3*h + c] for class c. */
+int vsa_plan_tile_counts(vsa_plan_t plan, int64_t* host_counts, size_t n, void* stream);
+
+/* Synchronous: perm[slot] = natural token index or -1 (padding), n >= n_slots. */
+int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream);
+
+/* Synchronous: number of executed (kv tile, 128-row query block) steps per
+ * head, host_dst[h]; the attention kernel runs one tensor-core tile per step. */
+int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream);
+
+/* Frees the plan's device buffers (synchronises the device first). */
+int vsa_plan_destroy(vsa_plan_t plan);
+
+/* Gather into tile-major order ([VDS] section 7.2: a [N,d] gather per head;
+ * [PSA] key design 2).  in: bf16 [B][num_heads][N][D] natural order;
+ * out: bf16 [B][num_heads][n_slots][D]; padding rows are written as zeros.
+ * D in {64,128}.  in and out must not overlap.  Asynchronous. */
+int vsa_permute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream);
+
+/* Restore natural order ([SVG-TPU], "supporting dynamic masks and token
+ * layouts": the order is restored after attention).  in: bf16
+ * [B][num_heads][n_slots][D]; out: bf16 [B][num_heads][N][D]; padding rows
+ * are dropped.  Asynchronous. */
+int vsa_unpermute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream);
+
+/* Block-sparse attention forward on tile-major tensors.
+ * q, k, v: bf16 [B][num_heads][n_slots][D]; o: bf16 same shape;
+ * lse: fp32 [B][num_heads][n_slots] (natural log of the sum over kept keys of
+ * exp(scale * q.k)).  For each real query row:
+ *   o_q = sum_{k kept} softmax_k(scale * q.k) v_k       ([STA] section 2, Eq. 1)
+ * Empty kv tiles are skipped, full tiles run with no per-element masking,
+ * boundary tiles evaluate the exact predicate, and partial results merge by
+ * online softmax ([SVG-TPU], "avoid in-tile masking when nothing needs
+ * masking").  A row with no kept key gets o = 0 and lse = -inf.  Padding rows
+ * of o and lse are unspecified.  D in {64,128}.  Asynchronous; device-side
+ * failures surface in vsa_check_status. */
+int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v,
+                        void* o, float* lse, vsa_plan_t plan,
+                        int B, int D, float scale, void* stream);
+
+/* Synchronises `stream`, then reports and clears the plan's device status
+ * word: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_DEVICE; VSA_ERR_CUDA if the
+ * stream itself failed. */
+int vsa_check_status(vsa_plan_t plan, void* stream);
+
+/* Static description of a status code. */
+const char* vsa_status_string(int code);
+
+/* VSA_VERSION of the built library. */
+int vsa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VSA_H */

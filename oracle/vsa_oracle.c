@@ -199,7 +199,8 @@ typedef struct {
     const orc_grid* g;
     int D;
     double scale;
-    const uint16_t *q, *k, *v;   /* [N, D] natural order, bf16 bits */
+    const uint16_t* q;           /* [N, D] natural order, bf16 bits */
+    const double *k, *v;         /* [N, D] natural order, widened to fp64 */
     const int64_t* rows;
     double* out_o;               /* [nrows, D] */
     double* out_lse;             /* [nrows] */
@@ -223,8 +224,8 @@ static void orc_attn_row(int64_t r, void* vctx)
         const int tk = (int)(nk / HW), hk = (int)((nk % HW) / c->g->W), wk = (int)(nk % c->g->W);
         if (!keep_coords(c->m, c->g, tq, hq, wq, tk, hk, wk)) { s[nk] = -INFINITY; continue; }
         double acc = 0.0;
-        const uint16_t* kr = c->k + nk * D;
-        for (int d = 0; d < D; ++d) acc += qd[d] * bf16_to_double(kr[d]);
+        const double* kr = c->k + nk * D;
+        for (int d = 0; d < D; ++d) acc += qd[d] * kr[d];
         s[nk] = acc * c->scale;
         if (s[nk] > mx) mx = s[nk];
     }
@@ -239,8 +240,8 @@ static void orc_attn_row(int64_t r, void* vctx)
         if (s[nk] == -INFINITY) continue;
         const double p = exp(s[nk] - mx);
         l += p;
-        const uint16_t* vr = c->v + nk * D;
-        for (int d = 0; d < D; ++d) o[d] += p * bf16_to_double(vr[d]);
+        const double* vr = c->v + nk * D;
+        for (int d = 0; d < D; ++d) o[d] += p * vr[d];
     }
     for (int d = 0; d < D; ++d) o[d] /= l;
     c->out_lse[r] = mx + log(l);
@@ -255,12 +256,19 @@ int orc_attention_rows(const orc_mask* m, const orc_grid* g, int D, double scale
 {
     if (!m || !g || !q || !k || !v || !rows || !out_o || !out_lse || D <= 0) return -1;
     orc_attn_ctx c;
-    c.m = m; c.g = g; c.D = D; c.scale = scale; c.q = q; c.k = k; c.v = v;
+    c.m = m; c.g = g; c.D = D; c.scale = scale; c.q = q;
     c.rows = rows; c.out_o = out_o; c.out_lse = out_lse;
     c.N = (int64_t)g->T * g->H * g->W;
     for (int64_t r = 0; r < nrows; ++r)
         if (rows[r] < 0 || rows[r] >= c.N) return -1;
+    /* bf16 -> fp64 is exact; widen k and v once */
+    double* kd = (double*)malloc(sizeof(double) * (size_t)c.N * D);
+    double* vd = (double*)malloc(sizeof(double) * (size_t)c.N * D);
+    if (!kd || !vd) { free(kd); free(vd); return -2; }
+    for (int64_t i = 0; i < c.N * D; ++i) { kd[i] = bf16_to_double(k[i]); vd[i] = bf16_to_double(v[i]); }
+    c.k = kd; c.v = vd;
     orc_parallel(nrows, nthreads, orc_attn_row, &c);
+    free(kd); free(vd);
     return 0;
 }
 

@@ -1,0 +1,102 @@
+"""Shared helpers for the GPU parity tests (test infrastructure).
+
+The CUDA path and the oracle only meet here: both consume the same seeded bf16
+inputs from ``workloads``, and their outputs are compared element by element.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import oracle
+import workloads as W
+
+# Output tolerance on N(0,1) inputs (max-abs and mean-abs against the fp64
+# oracle), and the lse tolerance.
+TOL_MAX = 2e-2
+TOL_MEAN = 2e-3
+TOL_LSE = 1e-2
+
+
+def torch_bf16(bits: np.ndarray):
+    import torch
+    t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+    return t.view(torch.bfloat16).cuda()
+
+
+def inverse_perm(perm: np.ndarray, n_tokens: int) -> np.ndarray:
+    inv = np.full(n_tokens, -1, dtype=np.int64)
+    real = perm >= 0
+    inv[perm[real]] = np.nonzero(real)[0]
+    assert (inv >= 0).all()
+    return inv
+
+
+class GpuRun:
+    """Run the whole path (plan, permute, forward, unpermute) on one workload."""
+
+    def __init__(self, w: W.Workload, inputs=None):
+        import torch
+        import block_sparse_attention_mask_b200 as vsa
+        self.w = w
+        self.grid = (w.T, w.H, w.W)
+        if inputs is None:
+            inputs = tuple(W.full_tensor(w, x) for x in "qkv")
+        self.q, self.k, self.v = inputs
+        self.plan = vsa.Plan(list(w.specs), self.grid, w.unit, w.q_tile, w.kv_tile)
+        qd, kd, vd = (torch_bf16(x) for x in (self.q, self.k, self.v))
+        o, lse = vsa.attention(self.plan, qd, kd, vd, scale=w.scale)
+        torch.cuda.synchronize()
+        self.plan.check()
+        del qd, kd, vd
+        self.o_dev = o                                  # natural order, on the GPU
+        self.lse_tm = lse.cpu().numpy().astype(np.float64)
+        self.perm = oracle.tile_major_order(self.grid, w.unit, self.plan.n_slots)
+        self.inv = inverse_perm(self.perm, w.N)
+
+    def o_rows(self, b: int, h: int, rows) -> np.ndarray:
+        import torch
+        idx = torch.as_tensor(np.asarray(rows, dtype=np.int64), device=self.o_dev.device)
+        return self.o_dev[b, h].index_select(0, idx).float().cpu().numpy().astype(np.float64)
+
+    def lse_natural(self, b: int, h: int) -> np.ndarray:
+        return self.lse_tm[b, h][self.inv]
+
+    def compare_rows(self, h: int, rows, b: int = 0):
+        """Oracle vs GPU on natural query rows of head h; returns (max, mean, lse max)."""
+        w = self.w
+        rows = np.asarray(rows, dtype=np.int64)
+        o_ref, lse_ref = oracle.attention_rows(w.specs[h], self.grid, w.unit, w.D, w.scale,
+                                               self.q[b, h], self.k[b, h], self.v[b, h], rows)
+        o_gpu = self.o_rows(b, h, rows)
+        lse_gpu = self.lse_natural(b, h)[rows]
+        assert np.isfinite(o_gpu).all(), "GPU output has non-finite values"
+        err = np.abs(o_gpu - o_ref)
+        fin = np.isfinite(lse_ref)
+        assert (np.isfinite(lse_gpu) == fin).all(), "rows with no kept key disagree"
+        assert (o_gpu[~fin] == 0).all()
+        lerr = float(np.abs(lse_gpu[fin] - lse_ref[fin]).max()) if fin.any() else 0.0
+        return float(err.max()), float(err.mean()), lerr
+
+    def check_rows(self, h: int, rows, b: int = 0):
+        mx, mean, lerr = self.compare_rows(h, rows, b)
+        assert mx <= TOL_MAX, f"head {h}: max abs err {mx}"
+        assert mean <= TOL_MEAN, f"head {h}: mean abs err {mean}"
+        assert lerr <= TOL_LSE, f"head {h}: lse max abs err {lerr}"
+        return mx, mean, lerr
+
+    def close(self):
+        self.plan.close()
+        self.o_dev = None
+
+
+def oracle_map_rows(w: W.Workload, h: int, n_slots: int, qtiles) -> np.ndarray:
+    return oracle.tile_map(w.specs[h], (w.T, w.H, w.W), w.unit, n_slots, w.q_tile, w.kv_tile,
+                           qtiles)
+
+
+def sample_qtiles(n_q: int, k: int, seed: int) -> np.ndarray:
+    g = np.random.default_rng(seed)
+    pick = {0, n_q - 1, n_q // 2}
+    while len(pick) < min(k, n_q):
+        pick.add(int(g.integers(0, n_q)))
+    return np.array(sorted(pick), dtype=np.int64)

@@ -1,0 +1,110 @@
+"""GPU parity at the full workload sizes, in the launch configuration the
+benchmark times (all heads, B = 1, the workload's tile shape).
+
+Outputs are compared with the oracle on stratified sampled rows (frame 0, last
+frame, the padded edge, corners, random), each row exact over all N keys.
+Tile maps are compared with the oracle's brute-force classes on sampled q-tile
+rows, and their per-head totals with closed forms where one exists.
+"""
+import numpy as np
+import pytest
+
+import workloads as W
+from _helpers import GpuRun, oracle_map_rows, sample_qtiles
+
+pytestmark = pytest.mark.gpu
+
+_INPUTS = {}
+
+
+def _inputs(w):
+    key = (w.T, w.H, w.W, w.heads, w.D, w.seeds)
+    if key not in _INPUTS:
+        _INPUTS.clear()
+        _INPUTS[key] = tuple(W.full_tensor(w, x) for x in "qkv")
+    return _INPUTS[key]
+
+
+def _check(w, heads, rows_per_head, map_heads, qtiles_per_head=6):
+    r = GpuRun(w, _inputs(w))
+    try:
+        errs = []
+        for h in heads:
+            errs.append(r.check_rows(h, W.sample_rows(w, h, rows_per_head)))
+        gmap = r.plan.tile_map()
+        for h in map_heads:
+            qt = sample_qtiles(gmap.shape[1], qtiles_per_head, seed=h)
+            ref = oracle_map_rows(w, h, r.plan.n_slots, qt)
+            assert (gmap[h][qt] == ref).all(), f"head {h}"
+        return r.plan.tile_counts(), errs
+    finally:
+        r.close()
+
+
+def _spatial_closed_form(T, Bq, Bk):
+    """Full / boundary tiles of one SVG spatial head (rt=1, sink) on T x 45 x 80.
+
+    (4T-4) kept frame pairs; per frame the q tiles and the kv tiles split into
+    those holding real rows only and those reaching the padded rows 45..47.
+    """
+    unit_w = 8 if min(Bq, Bk) == 64 else 16
+    units = 6 * (80 // unit_w)                 # units per padded frame
+    unit_tokens = 8 * unit_w
+    q_per_frame = units * unit_tokens // Bq
+    kv_per_frame = units * unit_tokens // Bk
+    kv_padded = (80 // unit_w) * unit_tokens // Bk if Bk >= unit_tokens else (80 // unit_w)
+    pairs = 4 * T - 4
+    return pairs * q_per_frame * (kv_per_frame - kv_padded), pairs * q_per_frame * kv_padded
+
+
+def test_tiny_all_rows():
+    w = W.tiny()
+    counts, _ = _check(w, range(w.heads), w.N, range(w.heads), qtiles_per_head=4)
+    assert counts.tolist() == [[4, 0, 12], [0, 12, 4]]
+
+
+def test_svg_wan720p():
+    w = W.svg_wan720p()
+    counts, _ = _check(w, range(w.heads), 96, [0, 7])
+    for h in range(5):
+        assert counts[h].tolist() == [324900, 12000, 60000]
+    for h in range(5, 10):
+        assert counts[h].tolist() == [290640, 90510, 15750]
+
+
+def test_sta_hunyuan720p():
+    w = W.sta_hunyuan720p()
+    counts, _ = _check(w, [0, 11, 23], 96, [0])
+    # 900 q tiles of 128 each see 45 window units x 3 tiles; no boundary tiles
+    for h in range(w.heads):
+        assert counts[h].tolist() == [810000 - 121500, 0, 121500]
+
+
+def test_stripe_wan720p():
+    w = W.stripe_wan720p()
+    counts, _ = _check(w, range(w.heads), 20, range(0, 40, 3), qtiles_per_head=4)
+    assert (counts.sum(axis=1) == 630 * 630).all()
+
+
+@pytest.mark.parametrize("T", W.SCALING_T)
+@pytest.mark.parametrize("mask", ["full", "spatial"])
+def test_scaling(T, mask):
+    w = W.scaling(T, mask)
+    counts, _ = _check(w, [0, 39], 48, [0])
+    n_tiles = (3840 * T // 128) ** 2
+    if mask == "full":
+        # only the kv tiles holding padded rows (5 of 30 per frame) are boundary
+        assert counts[0].tolist() == [0, n_tiles // 6, n_tiles - n_tiles // 6]
+    else:
+        full, bnd = _spatial_closed_form(T, 128, 128)
+        assert counts[0].tolist() == [n_tiles - full - bnd, bnd, full]
+
+
+@pytest.mark.parametrize("q_tile,kv_tile", [(q, k) for q in W.SWEEP_Q for k in W.SWEEP_KV
+                                            if (q, k) != (128, 128)])
+def test_tile_sweep(q_tile, kv_tile):
+    w = W.scaling(21, "spatial", q_tile, kv_tile)
+    counts, _ = _check(w, [0, 39], 48, [0])
+    full, bnd = _spatial_closed_form(21, q_tile, kv_tile)
+    assert counts[0][2] == full and counts[0][1] == bnd
+    assert bnd * 5 == full  # boundary share of executed tiles is 1/6

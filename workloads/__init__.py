@@ -204,13 +204,31 @@ def head_tensor(w: Workload, which: str, b: int, h: int) -> np.ndarray:
     return bf16_bits_from_f32(head_draw_f32(seed, b, h, w.N, w.D))
 
 
-def full_tensor(w: Workload, which: str, heads: Optional[Sequence[int]] = None) -> np.ndarray:
-    """bf16 bits [B, Hh, N, D] (natural order); only ``heads`` filled if given."""
+def full_tensor(w: Workload, which: str, heads: Optional[Sequence[int]] = None,
+                threads: Optional[int] = None) -> np.ndarray:
+    """bf16 bits [B, Hh, N, D] (natural order); only ``heads`` filled if given.
+
+    Heads are drawn in parallel threads; each head has its own stream, so the
+    result does not depend on the thread count.
+    """
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+
     out = np.zeros((w.B, w.heads, w.N, w.D), dtype=np.uint16)
-    hs = range(w.heads) if heads is None else heads
-    for b in range(w.B):
-        for h in hs:
-            out[b, h] = head_tensor(w, which, b, h)
+    hs = list(range(w.heads) if heads is None else heads)
+    jobs = [(b, h) for b in range(w.B) for h in hs]
+
+    def fill(job):
+        b, h = job
+        out[b, h] = head_tensor(w, which, b, h)
+
+    n = threads or min(len(jobs), os.cpu_count() or 1, 16)
+    if n <= 1:
+        for j in jobs:
+            fill(j)
+    else:
+        with ThreadPoolExecutor(n) as ex:
+            list(ex.map(fill, jobs))
     return out
 
 
