@@ -71,6 +71,7 @@ def _load() -> ctypes.CDLL:
         "vsa_plan_tile_counts": ([vp, vp, sz, vp], i32),
         "vsa_plan_perm": ([vp, vp, sz, vp], i32),
         "vsa_plan_exec_steps": ([vp, vp, sz, vp], i32),
+        "vsa_plan_kept_pairs": ([vp, vp, sz, vp], i32),
         "vsa_plan_destroy": ([vp], i32),
         "vsa_permute": ([vp, vp, vp, i32, i32, vp], i32),
         "vsa_unpermute": ([vp, vp, vp, i32, i32, vp], i32),
@@ -187,6 +188,14 @@ def vsa_plan_exec_steps(plan: int, stream=None) -> np.ndarray:
     return out
 
 
+def vsa_plan_kept_pairs(plan: int, stream=None) -> np.ndarray:
+    info = vsa_plan_info(plan)
+    out = np.empty(info["num_heads"], dtype=np.int64)
+    _check(_lib.vsa_plan_kept_pairs(plan, out.ctypes.data, out.size, _stream(stream)),
+           "vsa_plan_kept_pairs")
+    return out
+
+
 def vsa_plan_destroy(plan: int) -> None:
     _check(_lib.vsa_plan_destroy(plan), "vsa_plan_destroy")
 
@@ -259,6 +268,9 @@ class Plan:
 
     def exec_steps(self, stream=None) -> np.ndarray:
         return vsa_plan_exec_steps(self.handle, stream)
+
+    def kept_pairs(self, stream=None) -> np.ndarray:
+        return vsa_plan_kept_pairs(self.handle, stream)
 
     def check(self, stream=None) -> None:
         vsa_check_status(self.handle, stream)

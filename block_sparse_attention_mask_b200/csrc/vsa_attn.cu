@@ -247,54 +247,6 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
            ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-__device__ __forceinline__ uint32_t low_bits(int n) { return n >= 32 ? 0xFFFFFFFFu : ((1u << n) - 1u); }
-
-// Query-row context for the boundary predicate.
-struct RowCtx {
-    int tq, hq, wq, sq;
-    bool real;
-    int sta_t, sta_h, sta_w;   // first unit of the STA window per axis
-    int kk_t, kk_h, kk_w;      // window length per axis (clamped)
-};
-
-// Kept-key bits of one run of `nv` real keys at (t, h, w0 .. w0+nv-1).
-__device__ __forceinline__ uint32_t run_bits(const vsa_mask_spec& m, const vsa_dims& d, const RowCtx& q,
-                                             const uint32_t* stab, const uint32_t* ttab, int t, int h,
-                                             int w0, int nv)
-{
-    if (nv == 0 || !q.real) return 0u;
-    const uint32_t vm = low_bits(nv);
-    if (m.sink && t == 0) return vm;
-    switch (m.kind) {
-    case VSA_MASK_FULL:
-        return vm;
-    case VSA_MASK_SVG_SPATIAL:
-        return vsa_iabs(t - q.tq) <= m.rt ? vm : 0u;
-    case VSA_MASK_SVG_TEMPORAL: {
-        if (vsa_iabs(h - q.hq) > m.rh) return 0u;
-        const int lo = max(q.wq - m.rw, w0) - w0;
-        const int hi = min(q.wq + m.rw, w0 + nv - 1) - w0;
-        if (lo > hi) return 0u;
-        return low_bits(hi - lo + 1) << lo;
-    }
-    case VSA_MASK_STA: {
-        const int ut = t / d.bt, uh = h / d.bh, uw = w0 / d.bw;
-        const bool in = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h &&
-                        uh < q.sta_h + q.kk_h && uw >= q.sta_w && uw < q.sta_w + q.kk_w;
-        return in ? vm : 0u;
-    }
-    case VSA_MASK_STRIPE: {
-        const int it = t - q.tq + d.T - 1;
-        if (!((ttab[it >> 5] >> (it & 31)) & 1u)) return 0u;
-        const int x = h * d.W + w0 - q.sq + d.H * d.W - 1;
-        const uint32_t v = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31);
-        return v & vm;
-    }
-    default:
-        return 0u;
-    }
-}
-
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
 {
@@ -430,28 +382,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const int half = row >> 6;
         const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
         const vsa_mask_spec m = P.specs[head];
-        RowCtx q;
-        q.tq = q.hq = q.wq = 0;
-        q.real = vsa_slot_coords(d, (long long)e * kRows + row, q.tq, q.hq, q.wq);
-        q.sq = q.hq * d.W + q.wq;
-        q.kk_t = min(m.kt, d.nTt);
-        q.kk_h = min(m.kh, d.nTh);
-        q.kk_w = min(m.kw, d.nTw);
-        q.sta_t = vsa_sta_start(q.tq / d.bt, d.nTt, m.kt);
-        q.sta_h = vsa_sta_start(q.hq / d.bh, d.nTh, m.kh);
-        q.sta_w = vsa_sta_start(q.wq / d.bw, d.nTw, m.kw);
+        const vsa_row_ctx q = vsa_row_init(d, m, (long long)e * kRows + row);
         if (m.kind == VSA_MASK_STRIPE) {
             const uint32_t* src = P.sbits + (size_t)head * d.sbits_words;
             for (int i = row; i < P.tab_words_s; i += kRows) stab[i] = src[i];
-            for (int i = row; i < P.tab_words_t; i += kRows) {
-                uint32_t v = 0;
-                for (int b = 0; b < 32; ++b) {
-                    const int dt = i * 32 + b - (d.T - 1);
-                    if (dt > d.T - 1) break;
-                    if ((vsa_iabs(dt - m.To) % m.Ts) <= m.Tw - 1) v |= 1u << b;
-                }
-                ttab[i] = v;
-            }
+            for (int i = row; i < P.tab_words_t; i += kRows) ttab[i] = vsa_stripe_tword(m, d.T, i);
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
 
@@ -486,7 +421,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     uint32_t bits = 0;
                     for (int r = 0; r < runs_per_word; ++r) {
                         const int2 v = __ldg(sg + wi * runs_per_word + r);
-                        const uint32_t rb = run_bits(m, d, q, stab, ttab, v.x & 0xFFFF, v.x >> 16,
+                        const uint32_t rb = vsa_run_bits(m, d, q, stab, ttab, v.x & 0xFFFF, v.x >> 16,
                                                      v.y & 0xFFFF, v.y >> 16);
                         bits |= rb << (r * d.bw);
                     }
@@ -683,7 +618,7 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
     P.d = d;
     P.scale_log2 = scale * 1.4426950408889634f;
     P.tab_words_s = plan->has_stripe ? d.sbits_words : 0;
-    P.tab_words_t = plan->has_stripe ? (2 * d.T - 1 + 31) / 32 + 1 : 0;
+    P.tab_words_t = plan->has_stripe ? vsa_ttab_words(d.T) : 0;
 
     cudaStream_t s = (cudaStream_t)stream;
     if (D == 128 && d.Bk == 128) return launch_attn<128, 128>(P, B, s);

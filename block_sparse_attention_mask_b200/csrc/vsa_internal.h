@@ -107,4 +107,85 @@ __device__ __forceinline__ int vsa_sta_start(int uq, int n, int k)
     return s > n - kk ? n - kk : s;
 }
 
+__device__ __forceinline__ uint32_t vsa_low_bits(int n) { return n >= 32 ? 0xFFFFFFFFu : ((1u << n) - 1u); }
+
+// Query-row context for the boundary predicate.
+struct vsa_row_ctx {
+    int tq, hq, wq, sq;
+    bool real;
+    int sta_t, sta_h, sta_w;   // first unit of the STA window per axis
+    int kk_t, kk_h, kk_w;      // window length per axis (clamped)
+};
+
+// Kept-key bits of one run of `nv` real keys at (t, h, w0 .. w0+nv-1).
+__device__ __forceinline__ uint32_t vsa_run_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                             const uint32_t* stab, const uint32_t* ttab, int t, int h,
+                                             int w0, int nv)
+{
+    if (nv == 0 || !q.real) return 0u;
+    const uint32_t vm = vsa_low_bits(nv);
+    if (m.sink && t == 0) return vm;
+    switch (m.kind) {
+    case VSA_MASK_FULL:
+        return vm;
+    case VSA_MASK_SVG_SPATIAL:
+        return vsa_iabs(t - q.tq) <= m.rt ? vm : 0u;
+    case VSA_MASK_SVG_TEMPORAL: {
+        if (vsa_iabs(h - q.hq) > m.rh) return 0u;
+        const int lo = max(q.wq - m.rw, w0) - w0;
+        const int hi = min(q.wq + m.rw, w0 + nv - 1) - w0;
+        if (lo > hi) return 0u;
+        return vsa_low_bits(hi - lo + 1) << lo;
+    }
+    case VSA_MASK_STA: {
+        const int ut = t / d.bt, uh = h / d.bh, uw = w0 / d.bw;
+        const bool in = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h &&
+                        uh < q.sta_h + q.kk_h && uw >= q.sta_w && uw < q.sta_w + q.kk_w;
+        return in ? vm : 0u;
+    }
+    case VSA_MASK_STRIPE: {
+        const int it = t - q.tq + d.T - 1;
+        if (!((ttab[it >> 5] >> (it & 31)) & 1u)) return 0u;
+        const int x = h * d.W + w0 - q.sq + d.H * d.W - 1;
+        const uint32_t v = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31);
+        return v & vm;
+    }
+    default:
+        return 0u;
+    }
+}
+
+// Query-row context of tile-major slot `slot` for the predicate above.
+__device__ __forceinline__ vsa_row_ctx vsa_row_init(const vsa_dims& d, const vsa_mask_spec& m,
+                                                    long long slot)
+{
+    vsa_row_ctx q;
+    q.tq = q.hq = q.wq = 0;
+    q.real = vsa_slot_coords(d, slot, q.tq, q.hq, q.wq);
+    q.sq = q.hq * d.W + q.wq;
+    q.kk_t = min(m.kt, d.nTt);
+    q.kk_h = min(m.kh, d.nTh);
+    q.kk_w = min(m.kw, d.nTw);
+    q.sta_t = vsa_sta_start(q.tq / d.bt, d.nTt, m.kt);
+    q.sta_h = vsa_sta_start(q.hq / d.bh, d.nTh, m.kh);
+    q.sta_w = vsa_sta_start(q.wq / d.bw, d.nTw, m.kw);
+    return q;
+}
+
+// Word i of the stripe inter-frame table: bit b <-> dt = 32 i + b - (T - 1),
+// set when (|dt - To| mod Ts) <= Tw - 1 (dt = t_k - t_q).
+__device__ __forceinline__ uint32_t vsa_stripe_tword(const vsa_mask_spec& m, int T, int i)
+{
+    uint32_t v = 0;
+    for (int b = 0; b < 32; ++b) {
+        const int dt = i * 32 + b - (T - 1);
+        if (dt > T - 1) break;
+        if ((vsa_iabs(dt - m.To) % m.Ts) <= m.Tw - 1) v |= 1u << b;
+    }
+    return v;
+}
+
+// Words of the two stripe tables a kernel keeps in shared memory.
+static inline __host__ __device__ int vsa_ttab_words(int T) { return (2 * T - 1 + 31) / 32 + 1; }
+
 #endif  // __CUDACC__

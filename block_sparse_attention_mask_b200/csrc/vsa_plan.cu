@@ -314,6 +314,40 @@ __global__ void kv_list_kernel(vsa_dims d, const int8_t* __restrict__ map,
     }
 }
 
+// Kept (real query, real key) pairs per head: every real query row against
+// every run of keys of every kv tile, with the element predicate of the
+// boundary path.  One thread per query slot.
+__global__ void __launch_bounds__(256) kept_pairs_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                                         const uint32_t* __restrict__ sbits,
+                                                         const int2* __restrict__ seg,
+                                                         unsigned long long* __restrict__ kept)
+{
+    extern __shared__ uint32_t tabs[];
+    const int head = blockIdx.y;
+    const vsa_mask_spec m = specs[head];
+    const int ws = (m.kind == VSA_MASK_STRIPE) ? d.sbits_words : 0;
+    const int wt = (m.kind == VSA_MASK_STRIPE) ? vsa_ttab_words(d.T) : 0;
+    uint32_t* stab = tabs;
+    uint32_t* ttab = tabs + ws;
+    for (int i = threadIdx.x; i < ws; i += blockDim.x) stab[i] = sbits[(size_t)head * d.sbits_words + i];
+    for (int i = threadIdx.x; i < wt; i += blockDim.x) ttab[i] = vsa_stripe_tword(m, d.T, i);
+    __syncthreads();
+    const long long slot = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    unsigned long long cnt = 0;
+    if (slot < d.Npad) {
+        const vsa_row_ctx q = vsa_row_init(d, m, slot);
+        if (q.real) {
+            const long long nruns = (long long)d.nK * d.nseg;
+            for (long long r = 0; r < nruns; ++r) {
+                const int2 v = __ldg(seg + r);
+                cnt += __popc(vsa_run_bits(m, d, q, stab, ttab, v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16));
+            }
+        }
+    }
+    for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xFFFFFFFFu, cnt, off);
+    if ((threadIdx.x & 31) == 0 && cnt) atomicAdd(&kept[head], cnt);
+}
+
 __global__ void perm_kernel(vsa_dims d, int32_t* __restrict__ perm)
 {
     const long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -567,6 +601,32 @@ extern "C" int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n,
                                  cudaMemcpyDeviceToHost, s));
     VSA_CUDA_TRY(cudaStreamSynchronize(s));
     return VSA_OK;
+}
+
+extern "C" int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream)
+{
+    if (!plan || !host_dst || n < (size_t)plan->d.heads) return VSA_ERR_INVALID_ARG;
+    const vsa_dims& d = plan->d;
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned long long* tmp = nullptr;
+    if (cudaMalloc(&tmp, sizeof(unsigned long long) * d.heads) != cudaSuccess) {
+        cudaGetLastError();
+        return VSA_ERR_OOM;
+    }
+    const int smem = 4 * ((plan->has_stripe ? d.sbits_words : 0) + vsa_ttab_words(d.T));
+    cudaError_t e = cudaMemsetAsync(tmp, 0, sizeof(unsigned long long) * d.heads, s);
+    if (e == cudaSuccess && smem > 48 * 1024)
+        e = cudaFuncSetAttribute(kept_pairs_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess) {
+        dim3 g(blocks_for(d.Npad, 256), d.heads);
+        kept_pairs_kernel<<<g, 256, smem, s>>>(d, plan->d_specs, plan->d_sbits, plan->d_seg, tmp);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(host_dst, tmp, sizeof(unsigned long long) * d.heads, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    cudaFree(tmp);
+    return e == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 
 extern "C" int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream)

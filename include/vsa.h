@@ -154,6 +154,12 @@ int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream);
  * head, host_dst[h]; the attention kernel runs one tensor-core tile per step. */
 int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream);
 
+/* Synchronous: kept (real query, real key) pairs per head, host_dst[h]
+ * (the logical density the tile map approximates; [SVG-TPU], "logical
+ * sparsity is not physical sparsity").  Evaluates the element predicate on
+ * the GPU for every pair; allocates a small scratch buffer. */
+int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream);
+
 /* Frees the plan's device buffers (synchronises the device first). */
 int vsa_plan_destroy(vsa_plan_t plan);
 

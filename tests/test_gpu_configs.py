@@ -70,6 +70,12 @@ def test_svg_wan720p():
         assert counts[h].tolist() == [324900, 12000, 60000]
     for h in range(5, 10):
         assert counts[h].tolist() == [290640, 90510, 15750]
+    import block_sparse_attention_mask_b200 as vsa
+    plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile)
+    kept = plan.kept_pairs()
+    plan.close()
+    # spatial: 80 of 441 frame pairs; temporal: 21 sink frame pairs + 420 x 465 x 1288
+    assert kept.tolist() == [80 * 3600 ** 2] * 5 + [21 * 3600 ** 2 + 420 * 465 * 1288] * 5
 
 
 def test_sta_hunyuan720p():

@@ -133,3 +133,10 @@ def test_plan_rebuild_is_identical(run):
     run.plan.build()
     assert (run.plan.tile_map() == m1).all()
     assert (run.plan.tile_counts() == c1).all()
+
+
+def test_kept_pairs_match_oracle(run):
+    w = run.w
+    kept = run.plan.kept_pairs()
+    for h in range(w.heads):
+        assert int(kept[h]) == oracle.kept_pairs(w.specs[h], run.grid, w.unit), f"head {h}"
