@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "vsa_unpermute": ([vp, vp, vp, i32, i32, vp], i32),
         "vsa_sparse_attn_fwd": ([vp, vp, vp, vp, vp, vp, i32, i32, f32, vp], i32),
         "vsa_check_status": ([vp, vp], i32),
+        "vsa_tile_map_noalloc": ([P(vsa_mask_spec), i32, i32, i32, i32, i32, i32, i32, i32, i32, vp,
+                                  sz, vp], i32),
         "vsa_status_string": ([i32], ctypes.c_char_p),
         "vsa_version": ([], i32),
     }
@@ -214,6 +216,18 @@ def vsa_sparse_attn_fwd(q, k, v, o, lse, plan: int, B: int, D: int, scale: float
                         stream=None) -> None:
     _check(_lib.vsa_sparse_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), plan, int(B),
                                     int(D), float(scale), _stream(stream)), "vsa_sparse_attn_fwd")
+
+
+def vsa_tile_map_noalloc(specs: Sequence[Dict[str, int]], grid: Sequence[int], unit: Sequence[int],
+                         q_tile: int, kv_tile: int, map_out, stream=None) -> None:
+    """Tile map into a caller-owned int8 CUDA tensor; the library allocates nothing."""
+    arr = (vsa_mask_spec * len(specs))(*[make_spec(s) for s in specs])
+    T, H, W = (int(x) for x in grid)
+    bt, bh, bw = (int(x) for x in unit)
+    nbytes = map_out.numel() * map_out.element_size() if hasattr(map_out, "numel") else 0
+    _check(_lib.vsa_tile_map_noalloc(arr, len(specs), T, H, W, bt, bh, bw, int(q_tile), int(kv_tile),
+                                     _ptr(map_out), nbytes, _stream(stream)),
+           "vsa_tile_map_noalloc")
 
 
 def vsa_check_status(plan: int, stream=None) -> None:

@@ -58,6 +58,12 @@ struct vsa_plan_s {
     } while (0)
 
 int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s);
+int vsa_dims_for(int num_heads, int T, int H, int W, int bt, int bh, int bw, int q_tile, int kv_tile,
+                 int has_stripe, vsa_dims* out);
+int vsa_check_spec(const vsa_mask_spec* m);
+int vsa_launch_stripe_bits(const vsa_dims& d, const vsa_mask_spec* specs, uint32_t* sbits, cudaStream_t s);
+int vsa_launch_tile_map(const vsa_dims& d, const vsa_mask_spec* specs, const uint32_t* sbits, int8_t* map,
+                        cudaStream_t s);
 
 static inline bool vsa_aligned16(const void* p) { return (((uintptr_t)p) & 15u) == 0; }
 

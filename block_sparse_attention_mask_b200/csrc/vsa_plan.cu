@@ -558,6 +558,31 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     return VSA_OK;
 }
 
+// Launch helpers for other translation units (same kernels and launch shapes
+// as the plan build above).
+int vsa_dims_for(int num_heads, int T, int H, int W, int bt, int bh, int bw, int q_tile, int kv_tile,
+                 int has_stripe, vsa_dims* out)
+{
+    return compute_dims(num_heads, T, H, W, bt, bh, bw, q_tile, kv_tile, has_stripe, out);
+}
+
+int vsa_check_spec(const vsa_mask_spec* m) { return validate_spec(*m); }
+
+int vsa_launch_stripe_bits(const vsa_dims& d, const vsa_mask_spec* specs, uint32_t* sbits, cudaStream_t s)
+{
+    dim3 g(blocks_for(d.sbits_words, 128), d.heads);
+    stripe_bits_kernel<<<g, 128, 0, s>>>(d, specs, sbits);
+    return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
+int vsa_launch_tile_map(const vsa_dims& d, const vsa_mask_spec* specs, const uint32_t* sbits, int8_t* map,
+                        cudaStream_t s)
+{
+    const long long cells = (long long)d.heads * d.nQ * d.nK;
+    tile_map_kernel<<<blocks_for(cells, 256), 256, 0, s>>>(d, specs, sbits, map);
+    return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
+}
+
 extern "C" int vsa_plan_build(vsa_plan_t plan, void* stream)
 {
     if (!plan) return VSA_ERR_INVALID_ARG;

@@ -160,6 +160,35 @@ int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stre
  * the GPU for every pair; allocates a small scratch buffer. */
 int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream);
 
+/* No-allocation tile map.  None of the pages has a counterpart to this call;
+ * it serves callers that cannot call cudaMalloc: a host framework that owns
+ * all device memory through its own pool (a direct allocation would bypass
+ * its accounting and can fail once the pool holds the memory), or a serving
+ * loop that cannot afford cudaMalloc's implicit device synchronisation.
+ *
+ * Writes the same int8 map [num_heads][n_q_tiles][n_kv_tiles] that
+ * vsa_plan_create builds (arguments and supported shapes as there) into
+ * `map_out`, caller-owned device memory of `map_bytes` >= the map size
+ * (vsa_layout_info gives it).  Asynchronous on `stream`.
+ *
+ * Working memory is one file-scope device array of VSA_NOALLOC_SCRATCH_BYTES
+ * that every GPU loading the library holds until the process exits; it keeps
+ * the mask specs (at most VSA_NOALLOC_MAX_HEADS heads) and the stripe offset
+ * tables (4 * ceil((2*H*W - 1) / 32 + 1) bytes per head).  Larger requests
+ * fail with VSA_ERR_UNSUPPORTED before any device work.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ * The first call on a device looks up the array's device address with
+ * cudaGetSymbolAddress (once per device, with that device current); make that
+ * first call before any stream capture.  All calls share the array and it
+ * keeps the last call's contents (each call rewrites what it reads), so calls
+ * that overlap on the GPU race: serialise them, e.g. on one stream. */
+#define VSA_NOALLOC_SCRATCH_BYTES (1u << 20)
+#define VSA_NOALLOC_MAX_HEADS 64
+int vsa_tile_map_noalloc(const vsa_mask_spec* specs, int num_heads,
+                         int T, int H, int W, int bt, int bh, int bw,
+                         int q_tile, int kv_tile, int8_t* map_out, size_t map_bytes,
+                         void* stream);
+
 /* Frees the plan's device buffers (synchronises the device first). */
 int vsa_plan_destroy(vsa_plan_t plan);
 
