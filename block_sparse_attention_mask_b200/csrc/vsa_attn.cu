@@ -9,29 +9,28 @@
 // merge by online softmax ("Sparse VideoGen: accelerating video diffusion
 // attention on TPU", "avoid in-tile masking when nothing needs masking").
 //
-// One CTA = two consecutive 128-row query blocks X = 0, 1 of one (batch,
-// head); 12 warps in three warpgroups:
-//   warp 8      TMA producer: Q of both blocks once, then the K/V tiles of the
-//               merged (sorted) union of the two blocks' kv-tile lists through
-//               a STAGES-deep shared-memory ring; a tile both blocks list is
-//               loaded once and used by both.
-//   warp 9      MMA issuer (one thread): per block X, S_X = Q_X K^T into TMEM
-//               and O_X += P_X V with P_X read from TMEM (kind::f16, fp32
-//               accumulate).  Per block the order is PV(X, j-1), QK(X, j), so
-//               the tensor core alternates between the blocks while each
-//               block's softmax runs (ping-pong); tcgen05.commit signals the
-//               mbarriers.
-//   warps 10-11 idle (they complete the third warpgroup).
-//   warps 0..3  softmax of block 0, warps 4..7 softmax of block 1: thread r
-//               owns query row r (TMEM lane r).  It loads S, applies the
-//               boundary mask on boundary tiles, keeps the running max (log2
-//               units; O rescaled in TMEM only when the max grows by more than
-//               8, a factor 256) and sum in fp32, and writes P as bf16 over S
-//               in 32-column chunks; at the end it normalises O and writes o
-//               and lse.
-// Registers: launched at 168 per thread (384 x 168); the producer/MMA
-// warpgroup gives back down to 56 and the two softmax warpgroups take 224 each
-// (2 x 128 x 224 + 128 x 56 = 384 x 168), checked on the host before launch.
+// One CTA = one (batch, head, 128-row query block); 8 warps:
+//   warp 4      TMA producer: the K and V tiles of the block's kv-tile list
+//               through a STAGES-deep shared-memory ring (full/empty mbarriers).
+//   warp 5      MMA issuer (one thread).  Q sits in TMEM as the A operand, so
+//               S_j = Q K_j^T reads only K from shared memory; S is double
+//               buffered in TMEM, so QK_{j+1} runs while the softmax works on
+//               S_j; O += P_j V_j reads P_j from its own TMEM columns (no
+//               aliasing with S, so the tensor core never waits for a PV to
+//               drain before the next QK).  kind::f16, bf16 in, fp32
+//               accumulate; tcgen05.commit signals the mbarriers.
+//   warps 6, 7  mask workers: for every boundary tile of the list, thread t
+//               evaluates the exact predicate for rows t and t + 64 and stores
+//               the per-row keep bits in a shared-memory ring ahead of the
+//               softmax, so the softmax only applies them.
+//   warps 0..3  softmax: thread r owns query row r (TMEM lane r).  It first
+//               copies its Q row into TMEM, then per tile loads S_j, applies
+//               the exact predicate on boundary tiles only, keeps the running
+//               max (log2 units; O rescaled in TMEM only when the max grows by
+//               more than 8, a factor 256) and sum in fp32, and writes P_j as
+//               bf16; at the end it normalises O and writes o and lse.
+// TMEM columns: S0 [0,BK), S1 [BK,2BK), O [2BK,2BK+D), Q (D/2), P (BK/2):
+// 512 columns for D = BK = 128.
 // Every mbarrier wait is bounded: on expiry the CTA records VSA_DEV_TIMEOUT
 // in the plan's status word, all roles leave their loops, TMEM is freed and
 // the CTA exits.
@@ -39,41 +38,46 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
-#include <climits>
 #include <cstring>
 
 #include "vsa_internal.h"
 
 namespace {
 
-constexpr int kThreads = 384;
-constexpr int kLaunchRegs = 168;        // 65536 / 384, rounded down to a multiple of 8
-constexpr int kSoftmaxRegs = 224;
-constexpr int kControlRegs = 56;
-static_assert(2 * 128 * kSoftmaxRegs + 128 * kControlRegs <= kThreads * kLaunchRegs,
-              "register split exceeds the launch allocation");
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kRows = VSA_EXEC_ROWS;              // 128 query rows per block
+constexpr int kThreads = 256;
+constexpr int kProducerWarp = 4;
+constexpr int kMmaWarp = 5;
+constexpr int kMaskWarp0 = 6;                     // warps 6, 7
+constexpr int kMaskSlots = 4;                     // boundary-tile masks in flight
+constexpr int kRows = VSA_EXEC_ROWS;              // 128 query rows per CTA
 constexpr long long kWatchdogCycles = 1LL << 31;  // ~1 s at 2 GHz per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
+#ifndef VSA_POLY_EVERY
+#define VSA_POLY_EVERY 0                          // exp2 of every n-th column pair on the FMA pipe
+#endif
 
 template <int D, int BK>
 struct Cfg {
-    static constexpr int Q_BYTES = kRows * D * 2;   // one query block
     static constexpr int KV_BYTES = BK * D * 2;
-    static constexpr int STAGES = (2 * Q_BYTES + 4 * 2 * KV_BYTES <= 200 * 1024) ? 4
-                                  : (2 * Q_BYTES + 3 * 2 * KV_BYTES <= 200 * 1024) ? 3 : 2;
-    // TMEM: block X holds S_X (BK columns, P_X over its first BK/2) then O_X (D columns)
-    static constexpr int SPAN = BK + D;
-    static constexpr int TMEM_COLS = 2 * SPAN <= 256 ? 256 : 512;
+    static constexpr int STAGES = (4 * 2 * KV_BYTES <= 192 * 1024) ? 4 : (3 * 2 * KV_BYTES <= 192 * 1024) ? 3 : 2;
+    static constexpr int COL_S0 = 0;
+    static constexpr int COL_S1 = BK;
+    static constexpr int COL_O = 2 * BK;
+    static constexpr int COL_Q = 2 * BK + D;
+    static constexpr int COL_P = 2 * BK + D + D / 2;
+    static constexpr int COLS_USED = COL_P + BK / 2;
+    static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "TMEM budget");
     // shared memory map (offsets from a 1024-aligned base)
-    static constexpr int OFF_Q = 0;                 // block X at OFF_Q + X * Q_BYTES
-    static constexpr int OFF_K = 2 * Q_BYTES;
+    static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-    // barriers: q_full[2], k_full[S], v_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2]
-    static constexpr int NBAR = 2 + 3 * STAGES + 6;
+    // boundary masks: [slot][word][row] uint32, word = 32 key columns
+    static constexpr int OFF_MASK = OFF_V + STAGES * KV_BYTES;
+    static constexpr int MASK_SLOT_WORDS = (BK / 32) * kRows;
+    static constexpr int OFF_BAR = OFF_MASK + kMaskSlots * MASK_SLOT_WORDS * 4;
+    // barriers: k_full[S], v_full[S], kv_empty[S], s_full[2], p_full, pv_done, q_ready,
+    //           mask_full[M], mask_empty[M]
+    static constexpr int NBAR = 3 * STAGES + 5 + 2 * kMaskSlots;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem addr (4) + abort (4)
     static constexpr int OFF_TAB = (OFF_MISC + 8 + 15) / 16 * 16;
     // instruction descriptors (kind::f16): D fp32, A and B bf16
@@ -86,7 +90,8 @@ struct Cfg {
 };
 
 struct AttnParams {
-    CUtensorMap tm_q, tm_k, tm_v;       // 2D [rows = B*heads*n_slots, D] bf16, box {64, rows}
+    CUtensorMap tm_k, tm_v;             // 2D [rows = B*heads*n_slots, D] bf16, box {64, BK}
+    const __nv_bfloat16* q;
     __nv_bfloat16* o;
     float* lse;
     const int32_t* list_cnt;
@@ -257,6 +262,24 @@ __device__ __forceinline__ float ex2(float x)
     return y;
 }
 
+// 2^x on the FMA / ALU pipes, for x <= 8: Cody-Waite split x = n + f with
+// n = floor(x) (rounding-down add of 1.5 * 2^23 leaves n in the low mantissa
+// bits) and f in [0, 1); 2^f by the cubic 1 + c1 f + c2 f^2 + c3 f^3 fitted
+// here by minimax on the relative error with p(0) = 1, p(1) = 2 (linear
+// program on a dense grid; max relative error 1.03e-4, far below the 2^-9
+// rounding of the bf16 P it feeds); 2^n written into the exponent field.
+// x <= -127 (including -inf) gives exactly 0.
+__device__ __forceinline__ float ex2_poly(float x)
+{
+    x = fmaxf(x, -127.0f);
+    const float t = __fadd_rd(x, 12582912.0f);
+    const float n = t - 12582912.0f;
+    const float f = x - n;
+    const float p = fmaf(fmaf(fmaf(0.0782680781f, f, 0.226307771f), f, 0.695424151f), f, 1.0f);
+    const float scale = __int_as_float((__float_as_int(t) - (0x4B400000 - 127)) << 23);
+    return p * scale;
+}
+
 __device__ __forceinline__ float max3(float a, float b, float c)
 {
     float d;
@@ -304,24 +327,67 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
            ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Ordered union of two sorted kv-tile lists: each step yields the next kv
-// tile and which of the two lists hold it (bit X).
-struct ListMerge {
-    const int32_t* L[2];
-    int n[2];
-    int i[2];
-    __device__ __forceinline__ bool next(int& kv, int& mask)
-    {
-        const int a = i[0] < n[0] ? VSA_ENTRY_KV(__ldg(L[0] + i[0])) : INT_MAX;
-        const int b = i[1] < n[1] ? VSA_ENTRY_KV(__ldg(L[1] + i[1])) : INT_MAX;
-        if (a == INT_MAX && b == INT_MAX) return false;
-        kv = a < b ? a : b;
-        mask = (a == kv ? 1 : 0) | (b == kv ? 2 : 0);
-        i[0] += mask & 1;
-        i[1] += mask >> 1;
-        return true;
+// Mask-worker loop, specialised on the mask kind (uniform per CTA) so that
+// no per-run branch on the kind remains.  Thread t of the two mask warps
+// writes the keep bits of rows t and t + 64 for every boundary tile of the
+// list into slot (k mod kMaskSlots) of the ring, k = boundary tiles so far.
+// The run descriptors of a tile (bw keys sharing t and h each) are loaded
+// once per warp, one per lane, and broadcast with warp shuffles.
+template <int KIND, int BK>
+__device__ __forceinline__ void mask_worker_loop(const vsa_mask_spec& m_in, const vsa_dims& d,
+                                                 const vsa_row_ctx& q0, const vsa_row_ctx& q1,
+                                                 const uint32_t* stab, const uint32_t* ttab,
+                                                 const int2* __restrict__ seg, const int32_t* __restrict__ entries,
+                                                 int cnt, int t, int lane, uint32_t* maskbuf, uint32_t bar_mf0,
+                                                 uint32_t bar_me0, const Ctl& ctl)
+{
+    constexpr int MASK_SLOT_WORDS = (BK / 32) * kRows;
+    vsa_mask_spec m = m_in;
+    m.kind = KIND;                                  // lets the predicate's switch fold away
+    const int nseg = d.nseg;                        // BK / bw runs per tile, at most BK
+    const int bw = d.bw;
+    int kb = 0;
+    int ent_next = cnt > 0 ? __ldg(entries) : 0;
+    for (int j = 0; j < cnt; ++j) {
+        const int ent = ent_next;
+        if (j + 1 < cnt) ent_next = __ldg(entries + j + 1);
+        if (VSA_ENTRY_CLS(ent, 0) != VSA_TILE_BOUNDARY && VSA_ENTRY_CLS(ent, 1) != VSA_TILE_BOUNDARY) continue;
+        const int slot = kb % kMaskSlots;
+        const int2* sg = seg + (size_t)VSA_ENTRY_KV(ent) * nseg;
+        int2 rr[BK / 32];
+#pragma unroll
+        for (int i = 0; i < BK / 32; ++i) rr[i] = (i * 32 + lane < nseg) ? __ldg(sg + i * 32 + lane) : make_int2(0, 0);
+        if (kb >= kMaskSlots &&
+            !mbar_wait_warp(bar_me0 + 8u * slot, (uint32_t)(kb / kMaskSlots - 1) & 1, ctl))
+            return;
+        uint32_t* dst = maskbuf + slot * MASK_SLOT_WORDS;
+        uint32_t acc0 = 0, acc1 = 0;
+        for (int r = 0; r < nseg; ++r) {
+            const int src_reg = r >> 5;
+            int2 v = rr[0];
+#pragma unroll
+            for (int i = 1; i < BK / 32; ++i) v = (src_reg == i) ? rr[i] : v;
+            v.x = __shfl_sync(0xFFFFFFFFu, v.x, r & 31);
+            v.y = __shfl_sync(0xFFFFFFFFu, v.y, r & 31);
+            const int tt = v.x & 0xFFFF, hh = v.x >> 16, w0 = v.y & 0xFFFF, nv = v.y >> 16;
+            const uint32_t b0 = vsa_run_bits(m, d, q0, stab, ttab, tt, hh, w0, nv);
+            const uint32_t b1 = vsa_run_bits(m, d, q1, stab, ttab, tt, hh, w0, nv);
+            const int col = r * bw;                  // first key column of the run
+            const int sh = col & 31;                 // runs never straddle a word: bw divides 32
+            acc0 |= b0 << sh;
+            acc1 |= b1 << sh;
+            if (sh + bw == 32) {                     // last run of the 32-column word
+                dst[(col >> 5) * kRows + t] = acc0;
+                dst[(col >> 5) * kRows + t + 64] = acc1;
+                acc0 = 0;
+                acc1 = 0;
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_mf0 + 8u * slot);
+        ++kb;
     }
-};
+}
 
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
@@ -334,47 +400,48 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    const int npairs = (d.nE + 1) >> 1;
-    const int pair = blockIdx.x % npairs;
-    const int hb = blockIdx.x / npairs;                 // b * heads + head
+    const int e = blockIdx.x % d.nE;
+    const int hb = blockIdx.x / d.nE;                   // b * heads + head
     const int head = hb % d.heads;
     const long long base_row = (long long)hb * d.Nslots;
-    int eX[2], cnt[2];
-    const int32_t* list[2];
-#pragma unroll
-    for (int X = 0; X < 2; ++X) {
-        eX[X] = 2 * pair + X;
-        const bool present = eX[X] < d.nE;
-        const int li = head * d.nE + (present ? eX[X] : 0);
-        cnt[X] = present ? P.list_cnt[li] : 0;
-        list[X] = P.list + (size_t)li * d.nK;
-    }
+    const long long row0 = base_row + (long long)e * kRows;
+    const int list_idx = head * d.nE + e;
+    const int cnt = P.list_cnt[list_idx];
+    const int32_t* entries = P.list + (size_t)list_idx * d.nK;
 
     const uint32_t s_base = smem_addr(smem);
     const uint32_t bar0 = s_base + C::OFF_BAR;
-    auto BAR_Q = [&](int X) { return bar0 + 8u * X; };
-    auto BAR_KF = [&](int s) { return bar0 + 8u * (2 + s); };
-    auto BAR_VF = [&](int s) { return bar0 + 8u * (2 + C::STAGES + s); };
-    auto BAR_KE = [&](int s) { return bar0 + 8u * (2 + 2 * C::STAGES + s); };
-    auto BAR_SF = [&](int X) { return bar0 + 8u * (2 + 3 * C::STAGES + X); };
-    auto BAR_PF = [&](int X) { return bar0 + 8u * (4 + 3 * C::STAGES + X); };
-    auto BAR_OF = [&](int X) { return bar0 + 8u * (6 + 3 * C::STAGES + X); };
+    auto BAR_KF = [&](int s) { return bar0 + 8u * s; };
+    auto BAR_VF = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+    auto BAR_KE = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
+    auto BAR_SF = [&](int b) { return bar0 + 8u * (3 * C::STAGES + b); };
+    const uint32_t BAR_PF = bar0 + 8u * (3 * C::STAGES + 2);
+    const uint32_t BAR_PV = bar0 + 8u * (3 * C::STAGES + 3);
+    const uint32_t BAR_QR = bar0 + 8u * (3 * C::STAGES + 4);
+    auto BAR_MF = [&](int k) { return bar0 + 8u * (3 * C::STAGES + 5 + k); };
+    auto BAR_ME = [&](int k) { return bar0 + 8u * (3 * C::STAGES + 5 + kMaskSlots + k); };
+    uint32_t* maskbuf = (uint32_t*)(smem + C::OFF_MASK);
 
     uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
     volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
+    uint32_t* stab = (uint32_t*)(smem + C::OFF_TAB);
+    uint32_t* ttab = stab + P.tab_words_s;
     const Ctl ctl{abort_flag, P.status};
 
     if (threadIdx.x == 0) {
-        for (int X = 0; X < 2; ++X) {
-            mbar_init(BAR_Q(X), 1);
-            mbar_init(BAR_SF(X), 1);
-            mbar_init(BAR_PF(X), 4);
-            mbar_init(BAR_OF(X), 1);
-        }
         for (int s = 0; s < C::STAGES; ++s) {
             mbar_init(BAR_KF(s), 1);
             mbar_init(BAR_VF(s), 1);
             mbar_init(BAR_KE(s), 1);
+        }
+        mbar_init(BAR_SF(0), 1);
+        mbar_init(BAR_SF(1), 1);
+        mbar_init(BAR_PF, 4);
+        mbar_init(BAR_PV, 1);
+        mbar_init(BAR_QR, 4);
+        for (int k = 0; k < kMaskSlots; ++k) {
+            mbar_init(BAR_MF(k), 2);
+            mbar_init(BAR_ME(k), 4);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -392,26 +459,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // Each role starts with its setmaxnreg; every warp of a warpgroup executes
-    // the same one (warps 8..11 give registers back, warps 0..7 take them).
     if (warp == kProducerWarp) {
         // ---------------- TMA producer ----------------
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
         if (lane == 0) {
-#pragma unroll
-            for (int X = 0; X < 2; ++X) {
-                if (cnt[X] == 0) continue;
-                mbar_expect_tx(BAR_Q(X), C::Q_BYTES);
-                for (int c = 0; c < D / 64; ++c)
-                    tma_load_2d(s_base + C::OFF_Q + X * C::Q_BYTES + c * kRows * 128, &P.tm_q, c * 64,
-                                (int)(base_row + (long long)eX[X] * kRows), BAR_Q(X));
-            }
-            ListMerge mg{{list[0], list[1]}, {cnt[0], cnt[1]}, {0, 0}};
-            int kv, mask;
-            for (int u = 0; mg.next(kv, mask); ++u) {
-                const int st = u % C::STAGES;
-                const uint32_t use = (uint32_t)(u / C::STAGES);
-                if (u >= C::STAGES && !mbar_wait(BAR_KE(st), (use - 1) & 1, ctl)) break;
+            for (int j = 0; j < cnt; ++j) {
+                const int st = j % C::STAGES;
+                const uint32_t use = (uint32_t)(j / C::STAGES);
+                if (j >= C::STAGES && !mbar_wait(BAR_KE(st), (use - 1) & 1, ctl)) break;
+                const int kv = VSA_ENTRY_KV(__ldg(entries + j));
                 const int krow = (int)(base_row + (long long)kv * BK);
                 mbar_expect_tx(BAR_KF(st), C::KV_BYTES);
                 for (int c = 0; c < D / 64; ++c)
@@ -425,113 +480,126 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer ----------------
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
-        bool ok = true;
-        int pend_stage[2] = {-1, -1}, pend_item[2] = {0, 0}, nqk[2] = {0, 0}, npv[2] = {0, 0};
-        uint32_t users = 0;                      // per stage: 2-bit count of blocks still to run PV
-        bool qready[2] = {false, false};
-
-        auto issue_pv = [&](int X) -> bool {
-            const int st = pend_stage[X];
-            if (!mbar_wait_warp(BAR_PF(X), (uint32_t)(nqk[X] - 1) & 1, ctl)) return false;
-            if (!mbar_wait_warp(BAR_VF(st), (uint32_t)(pend_item[X] / C::STAGES) & 1, ctl)) return false;
+        // order: QK_0, QK_1, PV_0, QK_2, PV_1, ...; QK_{j+2} reuses S_{j%2},
+        // which the softmax finished reading before it signalled P_j
+        if (cnt > 0 && mbar_wait_warp(BAR_QR, 0, ctl)) {
             tc_fence_after();
-            if (lane == 0) {
-                const uint32_t aP = tmem + X * C::SPAN;
-                const uint32_t dO = tmem + X * C::SPAN + BK;
+            for (int j = 0; j <= cnt; ++j) {
+                if (j < cnt) {
+                    const int st = j % C::STAGES, b = j & 1;
+                    if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES) & 1, ctl)) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t dS = tmem + (b ? C::COL_S1 : C::COL_S0);
 #pragma unroll
-                for (int kk = 0; kk < BK / 16; ++kk) {
-                    const uint32_t va = s_base + C::OFF_V + st * C::KV_BYTES + kk * 16 * 128;
-                    mma_ts(dO, aP + kk * 8, smem_desc(va, BK * 128, 1024), C::IDESC_PV,
-                           (nqk[X] > 1 || kk > 0) ? 1u : 0u);
-                }
-            }
-            // O_X is complete after its last PV, wherever that PV is issued
-            // (a block whose list ended can get its last PV from the
-            // stage-release step below)
-            if (++npv[X] == cnt[X] && lane == 0) tc_commit(BAR_OF(X));
-            users -= 1u << (2 * st);
-            if (((users >> (2 * st)) & 3u) == 0 && lane == 0) tc_commit(BAR_KE(st));
-            __syncwarp();
-            pend_stage[X] = -1;
-            return true;
-        };
-
-        ListMerge mg{{list[0], list[1]}, {cnt[0], cnt[1]}, {0, 0}};
-        int kv, mask;
-        for (int u = 0; ok && mg.next(kv, mask); ++u) {
-            const int st = u % C::STAGES;
-            // PVs of the item that last used this stage must be issued before
-            // its K/V can be replaced
-#pragma unroll
-            for (int X = 0; X < 2; ++X)
-                if (ok && pend_stage[X] >= 0 && pend_item[X] <= u - C::STAGES) ok = issue_pv(X);
-            bool kready = false;
-#pragma unroll
-            for (int X = 0; X < 2; ++X) {
-                if (!ok || !((mask >> X) & 1)) continue;
-                // S_X is overwritten by QK(X): its previous P must be consumed first
-                if (pend_stage[X] >= 0) ok = issue_pv(X);
-                if (ok && !qready[X]) ok = qready[X] = mbar_wait_warp(BAR_Q(X), 0, ctl);
-                if (ok && !kready) {
-                    ok = kready = mbar_wait_warp(BAR_KF(st), (uint32_t)(u / C::STAGES) & 1, ctl);
-                    users |= (uint32_t)__popc(mask) << (2 * st);
-                }
-                if (!ok) break;
-                tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t dS = tmem + X * C::SPAN;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t qa = s_base + C::OFF_Q + X * C::Q_BYTES + (kk >> 2) * (kRows * 128) +
-                                            (kk & 3) * 32;
-                        const uint32_t ka = s_base + C::OFF_K + st * C::KV_BYTES + (kk >> 2) * (BK * 128) +
-                                            (kk & 3) * 32;
-                        mma_ss(dS, smem_desc(qa, 16, 1024), smem_desc(ka, 16, 1024), C::IDESC_QK,
-                               kk > 0 ? 1u : 0u);
+                        for (int kk = 0; kk < D / 16; ++kk) {
+                            const uint32_t ka = s_base + C::OFF_K + st * C::KV_BYTES + (kk >> 2) * (BK * 128) +
+                                                (kk & 3) * 32;
+                            mma_ts(dS, tmem + C::COL_Q + kk * 8, smem_desc(ka, 16, 1024), C::IDESC_QK,
+                                   kk > 0 ? 1u : 0u);
+                        }
+                        tc_commit(BAR_SF(b));
                     }
-                    tc_commit(BAR_SF(X));
+                    __syncwarp();
                 }
-                __syncwarp();
-                pend_stage[X] = st;
-                pend_item[X] = u;
-                ++nqk[X];
+                if (j >= 1) {
+                    const int jp = j - 1, stp = jp % C::STAGES;
+                    if (!mbar_wait_warp(BAR_PF, (uint32_t)jp & 1, ctl)) break;
+                    if (!mbar_wait_warp(BAR_VF(stp), (uint32_t)(jp / C::STAGES) & 1, ctl)) break;
+                    tc_fence_after();
+                    if (lane == 0) {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint32_t va = s_base + C::OFF_V + stp * C::KV_BYTES + kk * 16 * 128;
+                            mma_ts(tmem + C::COL_O, tmem + C::COL_P + kk * 8, smem_desc(va, BK * 128, 1024),
+                                   C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        tc_commit(BAR_PV);
+                        tc_commit(BAR_KE(stp));
+                    }
+                    __syncwarp();
+                }
             }
         }
-#pragma unroll
-        for (int X = 0; X < 2; ++X)
-            if (ok && pend_stage[X] >= 0) ok = issue_pv(X);
-    } else if (warp < 8) {
-        // ---------------- softmax: warps 4X .. 4X+3 own block X ----------------
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        const int X = warp >> 2;
-        const int row = threadIdx.x & 127;                // TMEM lane
-        const int half = row >> 6;
-        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + lane_off + X * C::SPAN;
-        const uint32_t tO = tS + BK;
+    } else if (warp >= kMaskWarp0) {
+        // ---------------- mask workers (warps 6, 7) ----------------
+        const int t = threadIdx.x - kMaskWarp0 * 32;      // rows t and t + 64
         const vsa_mask_spec m = P.specs[head];
-        const int n = cnt[X];
-        const vsa_row_ctx q = vsa_row_init(d, m, (long long)eX[X] * kRows + row);
-        uint32_t* stab = (uint32_t*)(smem + C::OFF_TAB) + X * (P.tab_words_s + P.tab_words_t);
-        uint32_t* ttab = stab + P.tab_words_s;
+        const vsa_row_ctx q0 = vsa_row_init(d, m, (long long)e * kRows + t);
+        const vsa_row_ctx q1 = vsa_row_init(d, m, (long long)e * kRows + t + 64);
         if (m.kind == VSA_MASK_STRIPE) {
             const uint32_t* src = P.sbits + (size_t)head * d.sbits_words;
-            for (int i = row; i < P.tab_words_s; i += kRows) stab[i] = src[i];
-            for (int i = row; i < P.tab_words_t; i += kRows) ttab[i] = vsa_stripe_tword(m, d.T, i);
+            for (int i = t; i < P.tab_words_s; i += 64) stab[i] = src[i];
         }
-        if (X == 0) asm volatile("bar.sync 1, 128;" ::: "memory");
-        else asm volatile("bar.sync 2, 128;" ::: "memory");
+        asm volatile("bar.sync 1, 192;" ::: "memory");
+        switch (m.kind) {
+        case VSA_MASK_FULL:
+            mask_worker_loop<VSA_MASK_FULL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane, maskbuf,
+                                                BAR_MF(0), BAR_ME(0), ctl);
+            break;
+        case VSA_MASK_SVG_SPATIAL:
+            mask_worker_loop<VSA_MASK_SVG_SPATIAL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane,
+                                                       maskbuf, BAR_MF(0), BAR_ME(0), ctl);
+            break;
+        case VSA_MASK_SVG_TEMPORAL:
+            mask_worker_loop<VSA_MASK_SVG_TEMPORAL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane,
+                                                        maskbuf, BAR_MF(0), BAR_ME(0), ctl);
+            break;
+        case VSA_MASK_STA:
+            mask_worker_loop<VSA_MASK_STA, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane, maskbuf,
+                                               BAR_MF(0), BAR_ME(0), ctl);
+            break;
+        default:
+            mask_worker_loop<VSA_MASK_STRIPE, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane,
+                                                  maskbuf, BAR_MF(0), BAR_ME(0), ctl);
+            break;
+        }
+    } else {
+        // ---------------- softmax warps 0..3 ----------------
+        const int row = threadIdx.x;                      // TMEM lane
+        const int half = row >> 6;
+        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        const uint32_t tO = tmem + lane_off + C::COL_O;
+        const uint32_t tP = tmem + lane_off + C::COL_P;
+        const vsa_mask_spec m = P.specs[head];
+        const vsa_row_ctx q = vsa_row_init(d, m, (long long)e * kRows + row);
+
+        // Q row -> TMEM (the QK operand), two bf16 per column
+        if (cnt > 0) {
+            const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row0 + row) * D);
+#pragma unroll
+            for (int c = 0; c < D / 64; ++c) {
+                uint32_t qv[32];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const uint4 x = __ldg(qrow + c * 8 + i);
+                    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
+                }
+                tmem_st32(tmem + lane_off + C::COL_Q + c * 32, qv);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR_QR);
+        }
+        if (m.kind == VSA_MASK_STRIPE)
+            for (int i = row; i < P.tab_words_t; i += kRows) ttab[i] = vsa_stripe_tword(m, d.T, i);
+        asm volatile("bar.sync 1, 192;" ::: "memory");
 
         float m_run = -INFINITY;  // running max of scale*log2(e)*s
         float l_run = 0.0f;
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
-        for (int j = 0; j < n && ok; ++j) {
-            const int ent = __ldg(list[X] + j);
+        int ent_next = cnt > 0 ? __ldg(entries) : 0;
+        int kb = 0;                                       // boundary tiles seen so far
+        for (int j = 0; j < cnt && ok; ++j) {
+            const int b = j & 1;
+            const int ent = ent_next;
+            if (j + 1 < cnt) ent_next = __ldg(entries + j + 1);
             const int cls = VSA_ENTRY_CLS(ent, half);
-            if (!mbar_wait_warp(BAR_SF(X), (uint32_t)j & 1, ctl)) { ok = false; break; }
+            const uint32_t tS = tmem + lane_off + (b ? C::COL_S1 : C::COL_S0);
+            if (!mbar_wait_warp(BAR_SF(b), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
             float s[BK];
             {
@@ -546,31 +614,32 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
 
-            if (cls == VSA_TILE_BOUNDARY) {
-                const int kv = VSA_ENTRY_KV(ent);
-                const int2* sg = P.seg + (size_t)kv * d.nseg;
-                const int runs_per_word = 32 / d.bw;
+            if (VSA_ENTRY_CLS(ent, 0) == VSA_TILE_BOUNDARY || VSA_ENTRY_CLS(ent, 1) == VSA_TILE_BOUNDARY) {
+                // keep bits from the mask workers; the slot is released after reading
+                const int slot = kb % kMaskSlots;
+                if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }
+                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + row;
+                uint32_t mw[BK / 32];
 #pragma unroll
-                for (int wi = 0; wi < BK / 32; ++wi) {
-                    uint32_t bits = 0;
-                    for (int r = 0; r < runs_per_word; ++r) {
-                        const int2 v = __ldg(sg + wi * runs_per_word + r);
-                        const uint32_t rb = vsa_run_bits(m, d, q, stab, ttab, v.x & 0xFFFF, v.x >> 16,
-                                                         v.y & 0xFFFF, v.y >> 16);
-                        bits |= rb << (r * d.bw);
-                    }
+                for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = src[wi * kRows];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR_ME(slot));
+                ++kb;
+                if (cls == VSA_TILE_BOUNDARY) {
 #pragma unroll
-                    for (int c = 0; c < 32; ++c)
-                        if (!((bits >> c) & 1u)) s[wi * 32 + c] = -INFINITY;
+                    for (int wi = 0; wi < BK / 32; ++wi)
+#pragma unroll
+                        for (int c = 0; c < 32; ++c)
+                            if (!((mw[wi] >> c) & 1u)) s[wi * 32 + c] = -INFINITY;
                 }
             }
 
+            uint32_t pk[BK / 2];
+            bool need_o = false;
+            float alpha = 1.0f;
             if (cls == VSA_TILE_EMPTY) {
-                uint32_t z[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i) z[i] = 0u;
-#pragma unroll
-                for (int c = 0; c < BK / 32; ++c) tmem_st16(tS + c * 16, z);
+                for (int c = 0; c < BK / 2; ++c) pk[c] = 0u;
             } else {
                 // row max: independent chains of 3-input max over 32 columns each
                 float mc[BK / 32];
@@ -585,8 +654,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
                 for (int g = 1; g < BK / 32; ++g) mx = fmaxf(mx, mc[g]);
                 const float mxs = mx * sl;
-                bool need_o = false;
-                float alpha = 1.0f;
                 if (mx != -INFINITY) {
                     if (m_run == -INFINITY) {
                         m_run = mxs;  // nothing accumulated for this row yet: O row is 0
@@ -597,39 +664,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                         need_o = true;
                     }
                 }
-                // O_X = P_X(<j) V is complete here: PV(X, j-1) was issued before
-                // QK(X, j), whose completion the s_full wait observed
-                if (__any_sync(0xFFFFFFFFu, need_o)) {
-#pragma unroll
-                    for (int c = 0; c < D / 32; ++c) {
-                        uint32_t ov[32];
-                        tmem_ld32(tO + c * 32, ov);
-                        tmem_ld_wait();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) {
-                            reg_fence(ov[i]);
-                            ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
-                        }
-                        tmem_st32(tO + c * 32, ov);
-                    }
-                }
                 const float mneg = (m_run == -INFINITY) ? 0.0f : -m_run;
                 const unsigned long long mneg2 = f2_pack(mneg, mneg);
                 unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int c = 0; c < BK / 32; ++c) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int k = c * 32 + 2 * i;
-                        float x0, x1;
-                        f2_unpack(f2_fma(f2_pack(s[k], s[k + 1]), sl2, mneg2), x0, x1);
-                        const float p0 = ex2(x0), p1 = ex2(x1);
-                        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-                        pk[i] = pack_bf16(p0, p1);
-                    }
-                    // P chunk c over S columns [16c, 16c+16): two bf16 per column
-                    tmem_st16(tS + c * 16, pk);
+                for (int i = 0; i < BK / 2; ++i) {
+                    float x0, x1;
+                    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2, mneg2), x0, x1);
+                    const bool poly = VSA_POLY_EVERY > 0 && (i % (VSA_POLY_EVERY > 0 ? VSA_POLY_EVERY : 1)) ==
+                                                                (VSA_POLY_EVERY > 0 ? VSA_POLY_EVERY - 1 : 0);
+                    const float p0 = poly ? ex2_poly(x0) : ex2(x0);
+                    const float p1 = poly ? ex2_poly(x1) : ex2(x1);
+                    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+                    pk[i] = pack_bf16(p0, p1);
                 }
                 float a0, a1, a2, a3, a4, a5, a6, a7;
                 f2_unpack(acc[0], a0, a1);
@@ -638,48 +685,65 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 f2_unpack(acc[3], a6, a7);
                 l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR_PF(X));
-        }
-
-        // ---------------- epilogue ----------------
-        if (eX[X] < d.nE) {
-            const long long orow = base_row + (long long)eX[X] * kRows + row;
-            bool have_o = ok && n > 0;
-            if (have_o) {
-                have_o = mbar_wait_warp(BAR_OF(X), 0, ctl);
+            // PV_{j-1} must be complete before P is overwritten and before O is
+            // rescaled; every phase of its barrier is awaited in order
+            if (j > 0) {
+                if (!mbar_wait_warp(BAR_PV, (uint32_t)(j - 1) & 1, ctl)) { ok = false; break; }
                 tc_fence_after();
             }
-            uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D);
-            if (have_o) {
-                const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            if (__any_sync(0xFFFFFFFFu, need_o)) {
 #pragma unroll
                 for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
                     tmem_ld32(tO + c * 32, ov);
                     tmem_ld_wait();
-                    uint32_t pkd[16];
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
+                    for (int i = 0; i < 32; ++i) {
                         reg_fence(ov[i]);
-                        reg_fence(ov[i + 1]);
-                        pkd[i >> 1] = pack_bf16(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                        ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                     }
-#pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        optr[c * 4 + i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+                    tmem_st32(tO + c * 32, ov);
                 }
-            } else {
-#pragma unroll
-                for (int i = 0; i < D / 8; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
             }
-            P.lse[orow] = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BK / 64; ++c) tmem_st32(tP + c * 32, pk + c * 32);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR_PF);
         }
-    } else {
-        // warps 10, 11: no work, but they belong to the control warpgroup
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+
+        // ---------------- epilogue ----------------
+        const long long orow = row0 + row;
+        bool have_o = ok && cnt > 0;
+        if (have_o) {
+            have_o = mbar_wait_warp(BAR_PV, (uint32_t)(cnt - 1) & 1, ctl);
+            tc_fence_after();
+        }
+        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D);
+        if (have_o) {
+            const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(tO + c * 32, ov);
+                tmem_ld_wait();
+                uint32_t pkd[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    reg_fence(ov[i]);
+                    reg_fence(ov[i + 1]);
+                    pkd[i >> 1] = pack_bf16(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    optr[c * 4 + i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        P.lse[orow] = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
 
     // ---------------- teardown ----------------
@@ -729,16 +793,12 @@ template <int D, int BK>
 int launch_attn(AttnParams& P, int B, cudaStream_t s)
 {
     using C = Cfg<D, BK>;
-    const int smem = 1024 + C::OFF_TAB + 2 * 4 * (P.tab_words_s + P.tab_words_t);
+    const int smem = 1024 + C::OFF_TAB + 4 * (P.tab_words_s + P.tab_words_t);
     if (smem > 227 * 1024) return VSA_ERR_UNSUPPORTED;
     auto kern = attn_fwd_kernel<D, BK>;
-    // the setmaxnreg split assumes exactly kLaunchRegs registers per thread at launch
-    cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return VSA_ERR_CUDA;
-    if (fa.numRegs != kLaunchRegs) return VSA_ERR_DEVICE;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return VSA_ERR_CUDA;
-    const long long grid = (long long)((P.d.nE + 1) / 2) * P.d.heads * B;
+    const long long grid = (long long)P.d.nE * P.d.heads * B;
     if (grid > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
     kern<<<(unsigned)grid, kThreads, smem, s>>>(P);
     return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
@@ -762,9 +822,8 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
 
     AttnParams P;
     memset(&P, 0, sizeof P);
-    if (!make_map(&P.tm_q, q, rows, D, kRows) || !make_map(&P.tm_k, k, rows, D, d.Bk) ||
-        !make_map(&P.tm_v, v, rows, D, d.Bk))
-        return VSA_ERR_CUDA;
+    if (!make_map(&P.tm_k, k, rows, D, d.Bk) || !make_map(&P.tm_v, v, rows, D, d.Bk)) return VSA_ERR_CUDA;
+    P.q = (const __nv_bfloat16*)q;
     P.o = (__nv_bfloat16*)o;
     P.lse = lse;
     P.list_cnt = plan->d_list_cnt;
