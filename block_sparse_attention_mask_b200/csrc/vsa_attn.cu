@@ -210,6 +210,17 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
         : "memory");
 }
 
+// Same, with the accumulate flag as an immediate (folded by ptxas).
+template <int ACC>
+__device__ __forceinline__ void mma_ts_i(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "n"(ACC)
+        : "memory");
+}
+
 // 32 lanes x 32 columns of 32 bit: thread i of the warp gets lane (base + i), columns c..c+31.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r)
 {
@@ -482,6 +493,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // ---------------- MMA issuer ----------------
         // order: QK_0, QK_1, PV_0, QK_2, PV_1, ...; QK_{j+2} reuses S_{j%2},
         // which the softmax finished reading before it signalled P_j
+        // Descriptors are built once; per MMA only a compile-time offset is
+        // added (the start-address field sits in the low bits and never carries).
+        const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
+        const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
+        constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
         if (cnt > 0 && mbar_wait_warp(BAR_QR, 0, ctl)) {
             tc_fence_after();
             for (int j = 0; j <= cnt; ++j) {
@@ -491,13 +507,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     tc_fence_after();
                     if (lane == 0) {
                         const uint32_t dS = tmem + (b ? C::COL_S1 : C::COL_S0);
+                        const uint32_t aQ = tmem + C::COL_Q;
+                        const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
+                        mma_ts_i<0>(dS, aQ, kd, C::IDESC_QK);
 #pragma unroll
-                        for (int kk = 0; kk < D / 16; ++kk) {
-                            const uint32_t ka = s_base + C::OFF_K + st * C::KV_BYTES + (kk >> 2) * (BK * 128) +
-                                                (kk & 3) * 32;
-                            mma_ts(dS, tmem + C::COL_Q + kk * 8, smem_desc(ka, 16, 1024), C::IDESC_QK,
-                                   kk > 0 ? 1u : 0u);
-                        }
+                        for (int kk = 1; kk < D / 16; ++kk)
+                            mma_ts_i<1>(dS, aQ + kk * 8,
+                                        kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
+                                        C::IDESC_QK);
                         tc_commit(BAR_SF(b));
                     }
                     __syncwarp();
@@ -508,12 +525,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     if (!mbar_wait_warp(BAR_VF(stp), (uint32_t)(jp / C::STAGES) & 1, ctl)) break;
                     tc_fence_after();
                     if (lane == 0) {
+                        const uint32_t dO = tmem + C::COL_O;
+                        const uint32_t aP = tmem + C::COL_P;
+                        const uint64_t vd = vdesc0 + (uint64_t)stp * kStageStep;
+                        if (jp == 0) mma_ts_i<0>(dO, aP, vd, C::IDESC_PV);
+                        else mma_ts_i<1>(dO, aP, vd, C::IDESC_PV);
 #pragma unroll
-                        for (int kk = 0; kk < BK / 16; ++kk) {
-                            const uint32_t va = s_base + C::OFF_V + stp * C::KV_BYTES + kk * 16 * 128;
-                            mma_ts(tmem + C::COL_O, tmem + C::COL_P + kk * 8, smem_desc(va, BK * 128, 1024),
-                                   C::IDESC_PV, (jp > 0 || kk > 0) ? 1u : 0u);
-                        }
+                        for (int kk = 1; kk < BK / 16; ++kk)
+                            mma_ts_i<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV);
                         tc_commit(BAR_PV);
                         tc_commit(BAR_KE(stp));
                     }
