@@ -135,6 +135,18 @@ def exec_flops(w, counts) -> float:
     return 4.0 * w.D * w.q_tile * w.kv_tile * executed
 
 
+def rank_workload(w, rank: int):
+    """The workload rank `rank` processes: same shape and masks, its own batch
+    element (independent seeds), so per-GPU work is fixed as ranks are added."""
+    return W.Workload(w.name, w.B, w.T, w.H, w.W, w.heads, w.D, w.unit, w.q_tile, w.kv_tile,
+                      w.specs, seeds=tuple(s + 1000 * rank for s in w.seeds))
+
+
+def aggregate_tflops(flops_per_rank_step: float, world: int, ms_max: float) -> float:
+    """Whole-job throughput: every rank's executed FLOPs over the slowest rank's step time."""
+    return flops_per_rank_step * world / (ms_max * 1e-3) / 1e12
+
+
 def dist_init():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -258,9 +270,8 @@ def run_gpu(args, w, world, rank, local):
     grid = (w.T, w.H, w.W)
     B = w.B
 
-    # inputs: rank r draws batch element r (weak scaling)
-    wr = W.Workload(w.name, w.B, w.T, w.H, w.W, w.heads, w.D, w.unit, w.q_tile, w.kv_tile,
-                    w.specs, seeds=tuple(s + 1000 * rank for s in w.seeds))
+    # inputs: rank r draws its own batch element (weak scaling)
+    wr = rank_workload(w, rank)
     host = [W.full_tensor(wr, x) for x in "qkv"]
     pinned = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in host]
     del host
@@ -333,7 +344,7 @@ def run_gpu(args, w, world, rank, local):
     ms_fwd = [a.elapsed_time(b) for a, b in fwd_events]
     ms_step = max_over_ranks(statistics.mean(ms_steps), world, dev)
     ms_fwd_mean = max_over_ranks(statistics.mean(ms_fwd), world, dev)
-    value = flops_step * world / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(flops_step, world, ms_step)
 
     # ---- end to end through the public API with host buffers ----
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
@@ -378,7 +389,7 @@ def run_gpu(args, w, world, rank, local):
     peak = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     achieved = flops_b * B / (ms_fwd_mean * 1e-3) / 1e12
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    prof = os.path.join(ROOT, "profiles", "attn_fwd_svg_wan720p_traffic.txt")
     if os.path.exists(prof):
         try:
             with open(prof) as f:
@@ -421,7 +432,7 @@ def run_gpu(args, w, world, rank, local):
                       "boundary_share_of_executed": float(counts[:, 1].sum() / max(1, counts[:, 1:].sum()))},
             "exec_steps": int(steps_exec.sum()),
             "cpu_baseline": cpu,
-            "e2e": {"value": flops_step * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+            "e2e": {"value": aggregate_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
                     "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clk,
             "gpu_launches": per_step_launches * args.steps,
@@ -456,11 +467,13 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     w = WORKLOADS[args.workload]()
+    if args.impl == "reference":
+        # the CPU oracle runs on rank 0 only; no process group is needed
+        run_reference(args, w, int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")))
+        return
     world, rank, local = dist_init()
     try:
-        if args.impl == "reference":
-            run_reference(args, w, world, rank)
-        else:
+        if True:
             res = run_gpu(args, w, world, rank, local)
             if rank == 0 and res is not None:
                 print(json.dumps(res), flush=True)

@@ -77,6 +77,7 @@ def _load() -> ctypes.CDLL:
         "vsa_unpermute": ([vp, vp, vp, i32, i32, vp], i32),
         "vsa_sparse_attn_fwd": ([vp, vp, vp, vp, vp, vp, i32, i32, f32, vp], i32),
         "vsa_check_status": ([vp, vp], i32),
+        "vsa_selftest_watchdog": ([vp, ctypes.c_longlong, vp], i32),
         "vsa_tile_map_noalloc": ([P(vsa_mask_spec), i32, i32, i32, i32, i32, i32, i32, i32, i32, vp,
                                   sz, vp], i32),
         "vsa_status_string": ([i32], ctypes.c_char_p),
@@ -232,6 +233,10 @@ def vsa_tile_map_noalloc(specs: Sequence[Dict[str, int]], grid: Sequence[int], u
 
 def vsa_check_status(plan: int, stream=None) -> None:
     _check(_lib.vsa_check_status(plan, _stream(stream)), "vsa_check_status")
+
+
+def vsa_selftest_watchdog(plan: int, cycles: int, stream=None) -> None:
+    _check(_lib.vsa_selftest_watchdog(plan, int(cycles), _stream(stream)), "vsa_selftest_watchdog")
 
 
 def vsa_status_string(code: int) -> str:

@@ -148,19 +148,24 @@ struct Ctl {
 };
 
 // Bounded wait for the phase of `bar` with the given parity to complete.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c)
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const Ctl& c, long long limit)
 {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
         if (mbar_try_wait(bar, parity)) return true;
         if (*c.abort) return false;
-        if (clock64() - t0 > kWatchdogCycles) {
+        if (clock64() - t0 > limit) {
             atomicOr(c.status, VSA_DEV_TIMEOUT);
             *c.abort = 1;
             return false;
         }
     }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Ctl& c)
+{
+    return mbar_wait_limit(bar, parity, c, kWatchdogCycles);
 }
 
 // Same, with the outcome made uniform across the warp (tcgen05.ld / st and
@@ -861,4 +866,34 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
     if (D == 128 && d.Bk == 64) return launch_attn<128, 64>(P, B, s);
     if (D == 64 && d.Bk == 128) return launch_attn<64, 128>(P, B, s);
     return launch_attn<64, 64>(P, B, s);
+}
+
+namespace {
+
+// One warp waits, with the attention kernel's bounded wait, on an mbarrier
+// that nothing arrives at; the wait expires after `limit` cycles and records
+// the timeout in the status word.
+__global__ void watchdog_selftest_kernel(unsigned int* status, long long limit)
+{
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ volatile int abort_flag;
+    const uint32_t b = smem_addr(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(b, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const Ctl ctl{&abort_flag, status};
+    if (threadIdx.x == 0) mbar_wait_limit(b, 0, ctl, limit);
+    __syncthreads();
+}
+
+}  // namespace
+
+extern "C" int vsa_selftest_watchdog(vsa_plan_t plan, long long cycles, void* stream)
+{
+    if (!plan || cycles <= 0 || cycles > kWatchdogCycles) return VSA_ERR_INVALID_ARG;
+    watchdog_selftest_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(plan->d_status, cycles);
+    return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }

@@ -224,6 +224,14 @@ int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v,
  * stream itself failed. */
 int vsa_check_status(vsa_plan_t plan, void* stream);
 
+/* Test hook for the device watchdog: launches one warp that waits, with the
+ * same bounded wait the attention kernel uses, on an mbarrier that nothing
+ * arrives at; after `cycles` SM clock cycles (1 .. 2^31) the wait gives up
+ * and records a timeout in the plan's status word, so the next
+ * vsa_check_status returns VSA_ERR_TIMEOUT and clears it.  Nothing faults,
+ * traps or hangs; the context stays usable.  Asynchronous. */
+int vsa_selftest_watchdog(vsa_plan_t plan, long long cycles, void* stream);
+
 /* Static description of a status code. */
 const char* vsa_status_string(int code);
 

@@ -85,6 +85,7 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_unpermute(None, None, None, 1, 128, None) == -1
     assert L.vsa_sparse_attn_fwd(None, None, None, None, None, None, 1, 128, 0.1, None) == -1
     assert L.vsa_check_status(None, None) == -1
+    assert L.vsa_selftest_watchdog(None, 1000, None) == -1
 
 
 def test_layout_slot_counts():
