@@ -369,7 +369,84 @@ __device__ __forceinline__ void mask_worker_loop(const vsa_mask_spec& m_in, cons
         if (j + 1 < cnt) ent_next = __ldg(entries + j + 1);
         if (VSA_ENTRY_CLS(ent, 0) != VSA_TILE_BOUNDARY && VSA_ENTRY_CLS(ent, 1) != VSA_TILE_BOUNDARY) continue;
         const int slot = kb % kMaskSlots;
-        const int2* sg = seg + (size_t)VSA_ENTRY_KV(ent) * nseg;
+        const int kv = VSA_ENTRY_KV(ent);
+        const int2* sg = seg + (size_t)kv * nseg;
+        if (d.box_nh > 0) {
+            // The tile is one box inside a unit: run r sits at t0 + r / box_nh,
+            // h0 + r % box_nh, with the same first column w0 and width for every
+            // run, so each run needs only a few operations per row.
+            const int2 v = __ldg(sg);
+            const int t0 = v.x & 0xFFFF, h0 = v.x >> 16, w0 = v.y & 0xFFFF;
+            const bool tile_real = (long long)kv * BK < d.Npad;
+            const int wv = tile_real ? max(0, min(bw, d.W - w0)) : 0;
+            const uint32_t vm = vsa_low_bits(wv);
+            if (kb >= kMaskSlots &&
+                !mbar_wait_warp(bar_me0 + 8u * slot, (uint32_t)(kb / kMaskSlots - 1) & 1, ctl))
+                return;
+            uint32_t* dst = maskbuf + slot * MASK_SLOT_WORDS;
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+                const vsa_row_ctx& q = which ? q1 : q0;
+                const int row = t + which * 64;
+                // row-invariant parts for this tile
+                uint32_t wmask = 0;             // temporal: kept w offsets of the run
+                bool sta_in = false;            // STA: the tile's unit is in the row's window
+                if (KIND == VSA_MASK_SVG_TEMPORAL) {
+                    const int lo = max(q.wq - m.rw, w0) - w0;
+                    const int hi = min(q.wq + m.rw, w0 + wv - 1) - w0;
+                    wmask = (lo <= hi) ? (vsa_low_bits(hi - lo + 1) << lo) : 0u;
+                }
+                if (KIND == VSA_MASK_STA) {
+                    const int ut = t0 / d.bt, uh = h0 / d.bh, uw = w0 / d.bw;
+                    sta_in = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h &&
+                             uh < q.sta_h + q.kk_h && uw >= q.sta_w && uw < q.sta_w + q.kk_w;
+                }
+                uint32_t acc = 0;
+                for (int r0 = 0; r0 < nseg; r0 += d.box_nh) {
+                    // one t-slice of the tile: everything but h is fixed here
+                    const int tt = t0 + r0 / d.box_nh;
+                    const bool tvalid = q.real && tt < d.T;
+                    const bool sinkhit = m.sink && tt == 0;
+                    bool tkeep = true;
+                    if (KIND == VSA_MASK_SVG_SPATIAL) tkeep = vsa_iabs(tt - q.tq) <= m.rt;
+                    if (KIND == VSA_MASK_STRIPE) {
+                        const int it = tt - q.tq + d.T - 1;
+                        tkeep = tvalid && ((ttab[it >> 5] >> (it & 31)) & 1u);
+                    }
+                    const int xbase = h0 * d.W + w0 - q.sq + d.H * d.W - 1;
+#pragma unroll 8
+                    for (int dh = 0; dh < d.box_nh; ++dh) {
+                        const int hh = h0 + dh;
+                        uint32_t b = 0;
+                        if (KIND == VSA_MASK_STRIPE) {
+                            const int x = xbase + dh * d.W;
+                            const uint32_t win = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31) & vm;
+                            b = (tkeep ? win : 0u);
+                        } else if (KIND == VSA_MASK_SVG_TEMPORAL) {
+                            b = vsa_iabs(hh - q.hq) <= m.rh ? wmask : 0u;
+                        } else if (KIND == VSA_MASK_SVG_SPATIAL) {
+                            b = tkeep ? vm : 0u;
+                        } else if (KIND == VSA_MASK_STA) {
+                            b = sta_in ? vm : 0u;
+                        } else {
+                            b = vm;
+                        }
+                        if (sinkhit) b = vm;
+                        if (!(tvalid && hh < d.H)) b = 0u;
+                        const int col = (r0 + dh) * bw;
+                        acc |= b << (col & 31);
+                        if (((col + bw) & 31) == 0) {
+                            dst[(col >> 5) * kRows + row] = acc;
+                            acc = 0;
+                        }
+                    }
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_mf0 + 8u * slot);
+            ++kb;
+            continue;
+        }
         int2 rr[BK / 32];
 #pragma unroll
         for (int i = 0; i < BK / 32; ++i) rr[i] = (i * 32 + lane < nseg) ? __ldg(sg + i * 32 + lane) : make_int2(0, 0);

@@ -30,6 +30,8 @@ struct vsa_dims {
     int nQ, nK;           // q tiles, kv tiles
     int nE;               // 128-row execution blocks
     int nseg;             // kv tile segments (Bk / bw)
+    int box_nh;           // when a kv tile is one box inside a unit: latent rows per t-slice
+                          // of the tile (its runs go h fastest, then t); 0 otherwise
     int sbits_words;      // words per head of the stripe offset table (0 if none)
     long long N, Npad, Nslots;
 };

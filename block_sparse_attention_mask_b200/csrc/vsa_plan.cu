@@ -468,6 +468,8 @@ static int compute_dims(int num_heads, int T, int H, int W, int bt, int bh, int 
     d.nK = (int)(d.Nslots / kv_tile);
     d.nE = (int)(d.Nslots / VSA_EXEC_ROWS);
     d.nseg = kv_tile / bw;
+    if (kv_tile <= d.U) d.box_nh = (kv_tile % (bh * bw) == 0) ? bh : kv_tile / bw;
+    else d.box_nh = 0;
     d.sbits_words = has_stripe ? (int)((2LL * H * W - 1 + 31) / 32 + 1) : 0;
     *out = d;
     return VSA_OK;
