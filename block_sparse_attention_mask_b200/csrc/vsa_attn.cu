@@ -9,26 +9,31 @@
 // merge by online softmax ("Sparse VideoGen: accelerating video diffusion
 // attention on TPU", "avoid in-tile masking when nothing needs masking").
 //
-// One CTA = one (batch, head, 128-row query block); 8 warps:
-//   warp 4      TMA producer: the K and V tiles of the block's kv-tile list
+// One CTA = one (batch, head, 128-row query block); 12 warps:
+//   warp 8      TMA producer: the K and V tiles of the block's kv-tile list
 //               through a STAGES-deep shared-memory ring (full/empty mbarriers).
-//   warp 5      MMA issuer (one thread).  Q sits in TMEM as the A operand, so
+//   warp 9      MMA issuer (one thread).  Q sits in TMEM as the A operand, so
 //               S_j = Q K_j^T reads only K from shared memory; S is double
 //               buffered in TMEM, so QK_{j+1} runs while the softmax works on
 //               S_j; O += P_j V_j reads P_j from its own TMEM columns (no
 //               aliasing with S, so the tensor core never waits for a PV to
 //               drain before the next QK).  kind::f16, bf16 in, fp32
 //               accumulate; tcgen05.commit signals the mbarriers.
-//   warps 6, 7  mask workers: for every boundary tile of the list, thread t
+//   warps 10,11 mask workers: for every boundary tile of the list, thread t
 //               evaluates the exact predicate for rows t and t + 64 and stores
 //               the per-row keep bits in a shared-memory ring ahead of the
 //               softmax, so the softmax only applies them.
-//   warps 0..3  softmax: thread r owns query row r (TMEM lane r).  It first
-//               copies its Q row into TMEM, then per tile loads S_j, applies
-//               the exact predicate on boundary tiles only, keeps the running
-//               max (log2 units; O rescaled in TMEM only when the max grows by
-//               more than 8, a factor 256) and sum in fp32, and writes P_j as
-//               bf16; at the end it normalises O and writes o and lse.
+//   warps 0..7  softmax, two warps per scheduler: warp w owns the 16 query
+//               rows (TMEM lanes) 32 (w mod 4) + 16 (w div 4) .. +15, and
+//               each row is split between lanes i and i + 16 of the warp,
+//               which hold the first and the second half of the row's columns
+//               (the 16x32bx2 TMEM access shape).  The pair combines its row
+//               max with one shuffle per tile; each half keeps its own partial
+//               row sum until the epilogue.  Per tile: load S_j, apply the keep
+//               bits on boundary tiles only, keep the running max (log2 units;
+//               O rescaled in TMEM only when the max grows by more than 8, a
+//               factor 256) and sum in fp32, and write P_j as bf16; at the end
+//               normalise O and write o and lse.
 // TMEM columns: S0 [0,BK), S1 [BK,2BK), O [2BK,2BK+D), Q (D/2), P (BK/2):
 // 512 columns for D = BK = 128.
 // Every mbarrier wait is bounded: on expiry the CTA records VSA_DEV_TIMEOUT
@@ -44,17 +49,15 @@
 
 namespace {
 
-constexpr int kThreads = 256;
-constexpr int kProducerWarp = 4;
-constexpr int kMmaWarp = 5;
-constexpr int kMaskWarp0 = 6;                     // warps 6, 7
+constexpr int kSoftmaxWarps = 8;                  // warps 0..7, two per scheduler
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kMaskWarp0 = 10;                    // warps 10, 11
+constexpr int kThreads = 32 * (kMaskWarp0 + 2);
 constexpr int kMaskSlots = 4;                     // boundary-tile masks in flight
 constexpr int kRows = VSA_EXEC_ROWS;              // 128 query rows per CTA
 constexpr long long kWatchdogCycles = 1LL << 31;  // ~1 s at 2 GHz per wait
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
-#ifndef VSA_POLY_EVERY
-#define VSA_POLY_EVERY 0                          // exp2 of every n-th column pair on the FMA pipe
-#endif
 
 template <int D, int BK>
 struct Cfg {
@@ -189,64 +192,60 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-__device__ __forceinline__ void tc_commit(uint32_t bar)
+// S or O += A B: A (M x 16) from TMEM, B from a shared-memory descriptor,
+// fp32 accumulate when ACC is 1.  Issued only by the lane whose `leader` is
+// nonzero; the operands are computed by the whole warp, so they stay
+// warp-uniform.
+template <int ACC>
+__device__ __forceinline__ void mma_ts_lead(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t leader)
 {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "n"(ACC), "r"(leader)
+        : "memory");
+}
+
+__device__ __forceinline__ void tc_commit_lead(uint32_t bar, uint32_t leader)
+{
+    asm volatile("{\n\t.reg .pred q;\n\tsetp.ne.b32 q, %1, 0;\n\t"
+                 "@q tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n"
+                 ::"r"(bar), "r"(leader)
                  : "memory");
 }
 
-__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accum)
+__device__ __forceinline__ uint32_t elect_one()
 {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accum)
-        : "memory");
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(r));
+    return r;
 }
 
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                       uint32_t accum)
+// 16 lanes x 2 column groups: thread i < 16 gets lane (base + i), columns
+// c..c+N-1; thread i >= 16 gets lane (base + i - 16), columns c+SPLIT..c+SPLIT+N-1.
+template <int SPLIT>
+__device__ __forceinline__ void tmem_ld_pair32(uint32_t taddr, uint32_t* r)
 {
     asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accum)
-        : "memory");
-}
-
-// Same, with the accumulate flag as an immediate (folded by ptxas).
-template <int ACC>
-__device__ __forceinline__ void mma_ts_i(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(bdesc), "r"(idesc), "n"(ACC)
-        : "memory");
-}
-
-// 32 lanes x 32 columns of 32 bit: thread i of the warp gets lane (base + i), columns c..c+31.
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r)
-{
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
           "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
+        : "r"(taddr), "n"(SPLIT));
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r)
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st_pair32(uint32_t taddr, const uint32_t* r)
 {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
+        "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr), "n"(SPLIT),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
@@ -255,14 +254,36 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r)
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r)
+template <int SPLIT>
+__device__ __forceinline__ void tmem_st_pair16(uint32_t taddr, const uint32_t* r)
 {
     asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
+        "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};" ::"r"(taddr), "n"(SPLIT),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
+}
+
+// A row half of W columns (W / 2 per thread, W / 2 >= 16) between registers and TMEM.
+template <int W>
+__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, uint32_t* r)
+{
+    static_assert(W % 64 == 0, "row halves are whole 32-column loads");
+#pragma unroll
+    for (int c = 0; c < W / 64; ++c) tmem_ld_pair32<W / 2>(taddr + c * 32, r + c * 32);
+}
+template <int W>
+__device__ __forceinline__ void tmem_st_half(uint32_t taddr, const uint32_t* r)
+{
+    static_assert(W % 32 == 0, "row halves are whole 16-column stores");
+    if constexpr (W % 64 == 0) {
+#pragma unroll
+        for (int c = 0; c < W / 64; ++c) tmem_st_pair32<W / 2>(taddr + c * 32, r + c * 32);
+    } else {
+#pragma unroll
+        for (int c = 0; c < W / 32; ++c) tmem_st_pair16<W / 2>(taddr + c * 16, r + c * 16);
+    }
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -276,24 +297,6 @@ __device__ __forceinline__ float ex2(float x)
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-// 2^x on the FMA / ALU pipes, for x <= 8: Cody-Waite split x = n + f with
-// n = floor(x) (rounding-down add of 1.5 * 2^23 leaves n in the low mantissa
-// bits) and f in [0, 1); 2^f by the cubic 1 + c1 f + c2 f^2 + c3 f^3 fitted
-// here by minimax on the relative error with p(0) = 1, p(1) = 2 (linear
-// program on a dense grid; max relative error 1.03e-4, far below the 2^-9
-// rounding of the bf16 P it feeds); 2^n written into the exponent field.
-// x <= -127 (including -inf) gives exactly 0.
-__device__ __forceinline__ float ex2_poly(float x)
-{
-    x = fmaxf(x, -127.0f);
-    const float t = __fadd_rd(x, 12582912.0f);
-    const float n = t - 12582912.0f;
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(0.0782680781f, f, 0.226307771f), f, 0.695424151f), f, 1.0f);
-    const float scale = __int_as_float((__float_as_int(t) - (0x4B400000 - 127)) << 23);
-    return p * scale;
 }
 
 __device__ __forceinline__ float max3(float a, float b, float c)
@@ -529,12 +532,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         mbar_init(BAR_SF(0), 1);
         mbar_init(BAR_SF(1), 1);
-        mbar_init(BAR_PF, 4);
+        mbar_init(BAR_PF, kSoftmaxWarps);
         mbar_init(BAR_PV, 1);
-        mbar_init(BAR_QR, 4);
+        mbar_init(BAR_QR, kSoftmaxWarps);
         for (int k = 0; k < kMaskSlots; ++k) {
             mbar_init(BAR_MF(k), 2);
-            mbar_init(BAR_ME(k), 4);
+            mbar_init(BAR_ME(k), kSoftmaxWarps);
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -573,57 +576,55 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer ----------------
-        // order: QK_0, QK_1, PV_0, QK_2, PV_1, ...; QK_{j+2} reuses S_{j%2},
-        // which the softmax finished reading before it signalled P_j
+        // The whole warp runs this role so that the descriptor and address
+        // arithmetic stays warp-uniform; one elected lane issues each
+        // tcgen05.mma and tcgen05.commit.
+        // Order: QK_0, QK_1, PV_0, QK_2, PV_1, ...; QK_{j+2} reuses S_{j%2},
+        // which the softmax finished reading before it signalled P_j.
         // Descriptors are built once; per MMA only a compile-time offset is
         // added (the start-address field sits in the low bits and never carries).
-        const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
-        const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
-        constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
+        const uint32_t leader = elect_one();
         if (cnt > 0 && mbar_wait_warp(BAR_QR, 0, ctl)) {
+            const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
+            const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
+            constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
+            const uint32_t aQ = tmem + C::COL_Q;
+            const uint32_t aP = tmem + C::COL_P;
+            const uint32_t dO = tmem + C::COL_O;
             tc_fence_after();
             for (int j = 0; j <= cnt; ++j) {
                 if (j < cnt) {
                     const int st = j % C::STAGES, b = j & 1;
                     if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES) & 1, ctl)) break;
                     tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t dS = tmem + (b ? C::COL_S1 : C::COL_S0);
-                        const uint32_t aQ = tmem + C::COL_Q;
-                        const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
-                        mma_ts_i<0>(dS, aQ, kd, C::IDESC_QK);
+                    const uint32_t dS = tmem + (b ? C::COL_S1 : C::COL_S0);
+                    const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
+                    mma_ts_lead<0>(dS, aQ, kd, C::IDESC_QK, leader);
 #pragma unroll
-                        for (int kk = 1; kk < D / 16; ++kk)
-                            mma_ts_i<1>(dS, aQ + kk * 8,
-                                        kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
-                                        C::IDESC_QK);
-                        tc_commit(BAR_SF(b));
-                    }
-                    __syncwarp();
+                    for (int kk = 1; kk < D / 16; ++kk)
+                        mma_ts_lead<1>(dS, aQ + kk * 8,
+                                       kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
+                                       C::IDESC_QK, leader);
+                    tc_commit_lead(BAR_SF(b), leader);
                 }
                 if (j >= 1) {
                     const int jp = j - 1, stp = jp % C::STAGES;
                     if (!mbar_wait_warp(BAR_PF, (uint32_t)jp & 1, ctl)) break;
                     if (!mbar_wait_warp(BAR_VF(stp), (uint32_t)(jp / C::STAGES) & 1, ctl)) break;
                     tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t dO = tmem + C::COL_O;
-                        const uint32_t aP = tmem + C::COL_P;
-                        const uint64_t vd = vdesc0 + (uint64_t)stp * kStageStep;
-                        if (jp == 0) mma_ts_i<0>(dO, aP, vd, C::IDESC_PV);
-                        else mma_ts_i<1>(dO, aP, vd, C::IDESC_PV);
+                    const uint64_t vd = vdesc0 + (uint64_t)stp * kStageStep;
+                    if (jp == 0) mma_ts_lead<0>(dO, aP, vd, C::IDESC_PV, leader);
+                    else mma_ts_lead<1>(dO, aP, vd, C::IDESC_PV, leader);
 #pragma unroll
-                        for (int kk = 1; kk < BK / 16; ++kk)
-                            mma_ts_i<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV);
-                        tc_commit(BAR_PV);
-                        tc_commit(BAR_KE(stp));
-                    }
-                    __syncwarp();
+                    for (int kk = 1; kk < BK / 16; ++kk)
+                        mma_ts_lead<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
+                    tc_commit_lead(BAR_PV, leader);
+                    tc_commit_lead(BAR_KE(stp), leader);
                 }
             }
         }
     } else if (warp >= kMaskWarp0) {
-        // ---------------- mask workers (warps 6, 7) ----------------
+        // ---------------- mask workers (warps 10, 11) ----------------
         const int t = threadIdx.x - kMaskWarp0 * 32;      // rows t and t + 64
         const vsa_mask_spec m = P.specs[head];
         const vsa_row_ctx q0 = vsa_row_init(d, m, (long long)e * kRows + t);
@@ -632,7 +633,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const uint32_t* src = P.sbits + (size_t)head * d.sbits_words;
             for (int i = t; i < P.tab_words_s; i += 64) stab[i] = src[i];
         }
-        asm volatile("bar.sync 1, 192;" ::: "memory");
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
         switch (m.kind) {
         case VSA_MASK_FULL:
             mask_worker_loop<VSA_MASK_FULL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane, maskbuf,
@@ -656,39 +657,42 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             break;
         }
     } else {
-        // ---------------- softmax warps 0..3 ----------------
-        const int row = threadIdx.x;                      // TMEM lane
-        const int half = row >> 6;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+        // ---------------- softmax warps 0..7 ----------------
+        // lanes i and i + 16 share query row (TMEM lane) rbase + i; hc picks
+        // the column half of S, P and O, and the keep-bit words, they hold.
+        const int rbase = 32 * (warp & 3) + 16 * (warp >> 2);
+        const int row = rbase + (lane & 15);
+        const int hc = lane >> 4;
+        const int half = row >> 6;                        // 64-row q tile of the row (warp-uniform)
+        const uint32_t lane_off = (uint32_t)rbase << 16;
         const uint32_t tO = tmem + lane_off + C::COL_O;
         const uint32_t tP = tmem + lane_off + C::COL_P;
         const vsa_mask_spec m = P.specs[head];
-        const vsa_row_ctx q = vsa_row_init(d, m, (long long)e * kRows + row);
 
-        // Q row -> TMEM (the QK operand), two bf16 per column
+        // Q row -> TMEM (the QK operand), two bf16 per column; each lane of
+        // the pair copies its half of the row
         if (cnt > 0) {
-            const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row0 + row) * D);
+            const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row0 + row) * D + hc * (D / 2));
+            uint32_t qv[D / 4];
 #pragma unroll
-            for (int c = 0; c < D / 64; ++c) {
-                uint32_t qv[32];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const uint4 x = __ldg(qrow + c * 8 + i);
-                    qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
-                }
-                tmem_st32(tmem + lane_off + C::COL_Q + c * 32, qv);
+            for (int i = 0; i < D / 16; ++i) {
+                const uint4 x = __ldg(qrow + i);
+                qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
             }
+            tmem_st_half<D / 2>(tmem + lane_off + C::COL_Q, qv);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR_QR);
         }
         if (m.kind == VSA_MASK_STRIPE)
-            for (int i = row; i < P.tab_words_t; i += kRows) ttab[i] = vsa_stripe_tword(m, d.T, i);
-        asm volatile("bar.sync 1, 192;" ::: "memory");
+            for (int i = threadIdx.x; i < P.tab_words_t; i += 32 * kSoftmaxWarps)
+                ttab[i] = vsa_stripe_tword(m, d.T, i);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
 
-        float m_run = -INFINITY;  // running max of scale*log2(e)*s
-        float l_run = 0.0f;
+        constexpr int NS = BK / 2;                        // S columns per lane
+        float m_run = -INFINITY;  // running max of scale*log2(e)*s (same in both lanes of the pair)
+        float l_run = 0.0f;       // partial row sum over this lane's columns
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
@@ -702,14 +706,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const uint32_t tS = tmem + lane_off + (b ? C::COL_S1 : C::COL_S0);
             if (!mbar_wait_warp(BAR_SF(b), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
-            float s[BK];
+            float s[NS];
             {
-                uint32_t sr[BK];
-#pragma unroll
-                for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+                uint32_t sr[NS];
+                tmem_ld_half<BK>(tS, sr);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < BK; ++c) {
+                for (int c = 0; c < NS; ++c) {
                     reg_fence(sr[c]);
                     s[c] = __uint_as_float(sr[c]);
                 }
@@ -719,33 +722,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 // keep bits from the mask workers; the slot is released after reading
                 const int slot = kb % kMaskSlots;
                 if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }
-                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + row;
-                uint32_t mw[BK / 32];
+                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + hc * (NS / 32) * kRows + row;
+                uint32_t mw[NS / 32];
 #pragma unroll
-                for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = src[wi * kRows];
+                for (int wi = 0; wi < NS / 32; ++wi) mw[wi] = src[wi * kRows];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR_ME(slot));
                 ++kb;
                 if (cls == VSA_TILE_BOUNDARY) {
 #pragma unroll
-                    for (int wi = 0; wi < BK / 32; ++wi)
+                    for (int wi = 0; wi < NS / 32; ++wi)
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
                             if (!((mw[wi] >> c) & 1u)) s[wi * 32 + c] = -INFINITY;
                 }
             }
 
-            uint32_t pk[BK / 2];
+            uint32_t pk[NS / 2];
             bool need_o = false;
             float alpha = 1.0f;
             if (cls == VSA_TILE_EMPTY) {
 #pragma unroll
-                for (int c = 0; c < BK / 2; ++c) pk[c] = 0u;
+                for (int c = 0; c < NS / 2; ++c) pk[c] = 0u;
             } else {
-                // row max: independent chains of 3-input max over 32 columns each
-                float mc[BK / 32];
+                // row max: independent chains of 3-input max over 32 columns
+                // each, then the other half of the row from the partner lane
+                float mc[NS / 32];
 #pragma unroll
-                for (int g = 0; g < BK / 32; ++g) {
+                for (int g = 0; g < NS / 32; ++g) {
                     float a = s[g * 32];
 #pragma unroll
                     for (int c = 1; c < 31; c += 2) a = max3(a, s[g * 32 + c], s[g * 32 + c + 1]);
@@ -753,7 +757,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
                 float mx = mc[0];
 #pragma unroll
-                for (int g = 1; g < BK / 32; ++g) mx = fmaxf(mx, mc[g]);
+                for (int g = 1; g < NS / 32; ++g) mx = fmaxf(mx, mc[g]);
+                mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
                 const float mxs = mx * sl;
                 if (mx != -INFINITY) {
                     if (m_run == -INFINITY) {
@@ -769,13 +774,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const unsigned long long mneg2 = f2_pack(mneg, mneg);
                 unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int i = 0; i < BK / 2; ++i) {
+                for (int i = 0; i < NS / 2; ++i) {
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2, mneg2), x0, x1);
-                    const bool poly = VSA_POLY_EVERY > 0 && (i % (VSA_POLY_EVERY > 0 ? VSA_POLY_EVERY : 1)) ==
-                                                                (VSA_POLY_EVERY > 0 ? VSA_POLY_EVERY - 1 : 0);
-                    const float p0 = poly ? ex2_poly(x0) : ex2(x0);
-                    const float p1 = poly ? ex2_poly(x1) : ex2(x1);
+                    const float p0 = ex2(x0);
+                    const float p1 = ex2(x1);
                     acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
                     pk[i] = pack_bf16(p0, p1);
                 }
@@ -794,20 +797,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
             if (__any_sync(0xFFFFFFFFu, need_o)) {
 #pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
+                for (int c = 0; c < D / 64; ++c) {
                     uint32_t ov[32];
-                    tmem_ld32(tO + c * 32, ov);
+                    tmem_ld_pair32<D / 2>(tO + c * 32, ov);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         reg_fence(ov[i]);
                         ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                     }
-                    tmem_st32(tO + c * 32, ov);
+                    tmem_st_pair32<D / 2>(tO + c * 32, ov);
                 }
             }
-#pragma unroll
-            for (int c = 0; c < BK / 64; ++c) tmem_st32(tP + c * 32, pk + c * 32);
+            tmem_st_half<BK / 2>(tP, pk);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
@@ -821,13 +823,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             have_o = mbar_wait_warp(BAR_PV, (uint32_t)(cnt - 1) & 1, ctl);
             tc_fence_after();
         }
-        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D);
+        const float l_row = l_run + __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
+        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D + hc * (D / 2));
         if (have_o) {
-            const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            const float inv = l_row > 0.0f ? 1.0f / l_row : 0.0f;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int c = 0; c < D / 64; ++c) {
                 uint32_t ov[32];
-                tmem_ld32(tO + c * 32, ov);
+                tmem_ld_pair32<D / 2>(tO + c * 32, ov);
                 tmem_ld_wait();
                 uint32_t pkd[16];
 #pragma unroll
@@ -842,9 +845,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < D / 8; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
+            for (int i = 0; i < D / 16; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
         }
-        P.lse[orow] = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        if (hc == 0)
+            P.lse[orow] = (l_row > 0.0f) ? (m_run + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
 
     // ---------------- teardown ----------------
