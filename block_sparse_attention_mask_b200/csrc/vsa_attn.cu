@@ -9,32 +9,39 @@
 // merge by online softmax ("Sparse VideoGen: accelerating video diffusion
 // attention on TPU", "avoid in-tile masking when nothing needs masking").
 //
-// One CTA = one (batch, head, 128-row query block); 12 warps:
-//   warp 8      TMA producer: the K and V tiles of the block's kv-tile list
-//               through a STAGES-deep shared-memory ring (full/empty mbarriers).
-//   warp 9      MMA issuer (one thread).  Q sits in TMEM as the A operand, so
-//               S_j = Q K_j^T reads only K from shared memory; S is double
-//               buffered in TMEM, so QK_{j+1} runs while the softmax works on
-//               S_j; O += P_j V_j reads P_j from its own TMEM columns (no
-//               aliasing with S, so the tensor core never waits for a PV to
-//               drain before the next QK).  kind::f16, bf16 in, fp32
-//               accumulate; tcgen05.commit signals the mbarriers.
+// One CTA = one (batch, head, 128-row query block).  The block's kv-tile list
+// is split between two softmax warpgroups by position: warpgroup X takes the
+// entries j with j mod 2 = X and keeps its own running max, running sum and
+// output accumulator O_X, so the two are independent streams that the tensor
+// core serves alternately; the epilogue merges the two partial softmaxes.  On
+// every scheduler one warp of each warpgroup runs, and as the two streams are
+// out of phase, one warp's exponentials (MUFU) overlap the other's loads,
+// masks and maxima.  12 warps:
+//   warp 8      TMA producer: lane 0 loads Q once and the K tiles of the list
+//               through a K ring, lane 1 the V tiles through a V ring
+//               (full/empty mbarriers per stage).
+//   warp 9      MMA issuer: the whole warp runs the loop so the descriptor
+//               arithmetic stays warp-uniform; one elected lane issues.
+//               S_j = Q K_j^T (both operands in shared memory) into S_{j mod 2};
+//               O_{j mod 2} += P_j V_j with P_j read from TMEM (it overwrites
+//               the first BK/2 columns of S_{j mod 2}) and V as an MN-major
+//               shared-memory operand.  kind::f16, bf16 in, fp32 accumulate;
+//               tcgen05.commit signals the mbarriers.  Issue order: QK_0,
+//               QK_1, PV_0, QK_2, PV_1, QK_3, ...; the tensor core runs one
+//               thread's MMAs in order, so by the time S_{j+2} is complete,
+//               PV_j has read P_j and finished accumulating into O_{j mod 2}.
 //   warps 10,11 mask workers: for every boundary tile of the list, thread t
 //               evaluates the exact predicate for rows t and t + 64 and stores
 //               the per-row keep bits in a shared-memory ring ahead of the
 //               softmax, so the softmax only applies them.
-//   warps 0..7  softmax, two warps per scheduler: warp w owns the 16 query
-//               rows (TMEM lanes) 32 (w mod 4) + 16 (w div 4) .. +15, and
-//               each row is split between lanes i and i + 16 of the warp,
-//               which hold the first and the second half of the row's columns
-//               (the 16x32bx2 TMEM access shape).  The pair combines its row
-//               max with one shuffle per tile; each half keeps its own partial
-//               row sum until the epilogue.  Per tile: load S_j, apply the keep
-//               bits on boundary tiles only, keep the running max (log2 units;
-//               O rescaled in TMEM only when the max grows by more than 8, a
-//               factor 256) and sum in fp32, and write P_j as bf16; at the end
-//               normalise O and write o and lse.
-// TMEM columns: S0 [0,BK), S1 [BK,2BK), O [2BK,2BK+D), Q (D/2), P (BK/2):
+//   warps 0..3  softmax warpgroup 0 and warps 4..7 warpgroup 1: thread r of a
+//               warpgroup owns query row r (TMEM lane r).  Per tile: load S_j,
+//               apply the keep bits on boundary tiles only, keep the running
+//               max (log2 units; O_X rescaled in TMEM only when the max grows
+//               by more than 8, a factor 256) and sum in fp32, and write P_j as
+//               bf16.  At the end both warpgroups merge their partial results
+//               and write o and lse, each half of the head dimension.
+// TMEM columns: S0 [0,BK), S1 [BK,2BK), O0 [2BK,2BK+D), O1 [2BK+D,2BK+2D):
 // 512 columns for D = BK = 128.
 // Every mbarrier wait is bounded: on expiry the CTA records VSA_DEV_TIMEOUT
 // in the plan's status word, all roles leave their loops, TMEM is freed and
@@ -49,11 +56,15 @@
 
 namespace {
 
-constexpr int kSoftmaxWarps = 8;                  // warps 0..7, two per scheduler
+constexpr int kSoftmaxWarps = 8;                  // warps 0..7: two warpgroups
 constexpr int kProducerWarp = 8;
 constexpr int kMmaWarp = 9;
 constexpr int kMaskWarp0 = 10;                    // warps 10, 11
 constexpr int kThreads = 32 * (kMaskWarp0 + 2);
+// Registers per thread: 168 at launch (65536 / 384 rounded down to 8); the
+// softmax warpgroups raise theirs with setmaxnreg and the third warpgroup
+// (producer, MMA, mask workers) gives the difference back.
+constexpr int kRegsLaunch = 168;
 constexpr int kMaskSlots = 4;                     // boundary-tile masks in flight
 constexpr int kRows = VSA_EXEC_ROWS;              // 128 query rows per CTA
 constexpr long long kWatchdogCycles = 1LL << 31;  // ~1 s at 2 GHz per wait
@@ -62,25 +73,37 @@ constexpr float kRescaleThreshold = 8.0f;         // log2 units
 template <int D, int BK>
 struct Cfg {
     static constexpr int KV_BYTES = BK * D * 2;
-    static constexpr int STAGES = (4 * 2 * KV_BYTES <= 192 * 1024) ? 4 : (3 * 2 * KV_BYTES <= 192 * 1024) ? 3 : 2;
+    static constexpr int Q_BYTES = kRows * D * 2;
+    // a softmax thread holds a whole S row (BK values) and its bf16 P
+    static constexpr int REGS_SOFTMAX = BK == 128 ? 208 : 176;
+    static constexpr int REGS_OTHER = 3 * kRegsLaunch - 2 * REGS_SOFTMAX;
+    static_assert(REGS_OTHER >= 24 && REGS_OTHER % 8 == 0, "setmaxnreg split");
+    static constexpr int RING_BYTES = 192 * 1024 - Q_BYTES;
+    // K stages are refilled once QK_j completes, V stages only once PV_j
+    // does, so K gets the deeper ring
+    static constexpr int STAGES_V = (RING_BYTES / KV_BYTES) / 2 > 4 ? 4 : (RING_BYTES / KV_BYTES) / 2;
+    static constexpr int STAGES_K = (RING_BYTES / KV_BYTES - STAGES_V) > 4 ? 4 : (RING_BYTES / KV_BYTES - STAGES_V);
+    static_assert(STAGES_V >= 2 && STAGES_K >= 2, "shared-memory ring");
     static constexpr int COL_S0 = 0;
     static constexpr int COL_S1 = BK;
-    static constexpr int COL_O = 2 * BK;
-    static constexpr int COL_Q = 2 * BK + D;
-    static constexpr int COL_P = 2 * BK + D + D / 2;
-    static constexpr int COLS_USED = COL_P + BK / 2;
+    static constexpr int COL_O0 = 2 * BK;
+    static constexpr int COL_O1 = 2 * BK + D;
+    static constexpr int COLS_USED = 2 * BK + 2 * D;
     static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM budget");
     // shared memory map (offsets from a 1024-aligned base)
-    static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + Q_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES_K * KV_BYTES;
     // boundary masks: [slot][word][row] uint32, word = 32 key columns
-    static constexpr int OFF_MASK = OFF_V + STAGES * KV_BYTES;
+    static constexpr int OFF_MASK = OFF_V + STAGES_V * KV_BYTES;
     static constexpr int MASK_SLOT_WORDS = (BK / 32) * kRows;
-    static constexpr int OFF_BAR = OFF_MASK + kMaskSlots * MASK_SLOT_WORDS * 4;
-    // barriers: k_full[S], v_full[S], kv_empty[S], s_full[2], p_full, pv_done, q_ready,
-    //           mask_full[M], mask_empty[M]
-    static constexpr int NBAR = 3 * STAGES + 5 + 2 * kMaskSlots;
+    // per-warpgroup row statistics (running max, running sum) for the merge
+    static constexpr int OFF_STAT = OFF_MASK + kMaskSlots * MASK_SLOT_WORDS * 4;
+    static constexpr int OFF_BAR = OFF_STAT + 2 * kRows * 8;
+    // barriers: k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], q_full,
+    //           s_full[2], p_full[2], pv_done[2], mask_full[M], mask_empty[M]
+    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 7 + 2 * kMaskSlots;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem addr (4) + abort (4)
     static constexpr int OFF_TAB = (OFF_MISC + 8 + 15) / 16 * 16;
     // instruction descriptors (kind::f16): D fp32, A and B bf16
@@ -93,8 +116,7 @@ struct Cfg {
 };
 
 struct AttnParams {
-    CUtensorMap tm_k, tm_v;             // 2D [rows = B*heads*n_slots, D] bf16, box {64, BK}
-    const __nv_bfloat16* q;
+    CUtensorMap tm_q, tm_k, tm_v;       // 2D [rows = B*heads*n_slots, D] bf16, box {64, 128 | BK}
     __nv_bfloat16* o;
     float* lse;
     const int32_t* list_cnt;
@@ -192,7 +214,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// S or O += A B: A (M x 16) from TMEM, B from a shared-memory descriptor,
+// S += A B with both operands in shared memory (descriptors), fp32
+// accumulate when ACC is 1; issued only by the lane whose `leader` is nonzero.
+template <int ACC>
+__device__ __forceinline__ void mma_ss_lead(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t leader)
+{
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\tsetp.ne.b32 p, %4, 0;\n\tsetp.ne.b32 q, %5, 0;\n\t"
+        "@q tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(idesc), "n"(ACC), "r"(leader)
+        : "memory");
+}
+
+// O += A B: A (M x 16) from TMEM, B from a shared-memory descriptor,
 // fp32 accumulate when ACC is 1.  Issued only by the lane whose `leader` is
 // nonzero; the operands are computed by the whole warp, so they stay
 // warp-uniform.
@@ -222,68 +257,33 @@ __device__ __forceinline__ uint32_t elect_one()
     return r;
 }
 
-// 16 lanes x 2 column groups: thread i < 16 gets lane (base + i), columns
-// c..c+N-1; thread i >= 16 gets lane (base + i - 16), columns c+SPLIT..c+SPLIT+N-1.
-template <int SPLIT>
-__device__ __forceinline__ void tmem_ld_pair32(uint32_t taddr, uint32_t* r)
+// 32 lanes x 32 columns of 32 bit: thread i of the warp gets lane (base + i), columns c..c+31.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r)
 {
     asm volatile(
-        "tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
         "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], %33;"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
           "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
           "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
           "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
           "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr), "n"(SPLIT));
+        : "r"(taddr));
 }
 
-template <int SPLIT>
-__device__ __forceinline__ void tmem_st_pair32(uint32_t taddr, const uint32_t* r)
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r)
 {
     asm volatile(
-        "tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], %1, "
-        "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33};" ::"r"(taddr), "n"(SPLIT),
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
         "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
         "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
         "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
         "r"(r[29]), "r"(r[30]), "r"(r[31])
         : "memory");
-}
-
-template <int SPLIT>
-__device__ __forceinline__ void tmem_st_pair16(uint32_t taddr, const uint32_t* r)
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], %1, "
-        "{%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17};" ::"r"(taddr), "n"(SPLIT),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-        : "memory");
-}
-
-// A row half of W columns (W / 2 per thread, W / 2 >= 16) between registers and TMEM.
-template <int W>
-__device__ __forceinline__ void tmem_ld_half(uint32_t taddr, uint32_t* r)
-{
-    static_assert(W % 64 == 0, "row halves are whole 32-column loads");
-#pragma unroll
-    for (int c = 0; c < W / 64; ++c) tmem_ld_pair32<W / 2>(taddr + c * 32, r + c * 32);
-}
-template <int W>
-__device__ __forceinline__ void tmem_st_half(uint32_t taddr, const uint32_t* r)
-{
-    static_assert(W % 32 == 0, "row halves are whole 16-column stores");
-    if constexpr (W % 64 == 0) {
-#pragma unroll
-        for (int c = 0; c < W / 64; ++c) tmem_st_pair32<W / 2>(taddr + c * 32, r + c * 32);
-    } else {
-#pragma unroll
-        for (int c = 0; c < W / 32; ++c) tmem_st_pair16<W / 2>(taddr + c * 16, r + c * 16);
-    }
 }
 
 __device__ __forceinline__ void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -508,15 +508,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t s_base = smem_addr(smem);
     const uint32_t bar0 = s_base + C::OFF_BAR;
     auto BAR_KF = [&](int s) { return bar0 + 8u * s; };
-    auto BAR_VF = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
-    auto BAR_KE = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
-    auto BAR_SF = [&](int b) { return bar0 + 8u * (3 * C::STAGES + b); };
-    const uint32_t BAR_PF = bar0 + 8u * (3 * C::STAGES + 2);
-    const uint32_t BAR_PV = bar0 + 8u * (3 * C::STAGES + 3);
-    const uint32_t BAR_QR = bar0 + 8u * (3 * C::STAGES + 4);
-    auto BAR_MF = [&](int k) { return bar0 + 8u * (3 * C::STAGES + 5 + k); };
-    auto BAR_ME = [&](int k) { return bar0 + 8u * (3 * C::STAGES + 5 + kMaskSlots + k); };
+    auto BAR_KE = [&](int s) { return bar0 + 8u * (C::STAGES_K + s); };
+    auto BAR_VF = [&](int s) { return bar0 + 8u * (2 * C::STAGES_K + s); };
+    auto BAR_VE = [&](int s) { return bar0 + 8u * (2 * C::STAGES_K + C::STAGES_V + s); };
+    constexpr int B1 = 2 * C::STAGES_K + 2 * C::STAGES_V;
+    const uint32_t BAR_QF = bar0 + 8u * B1;
+    auto BAR_SF = [&](int x) { return bar0 + 8u * (B1 + 1 + x); };
+    auto BAR_PF = [&](int x) { return bar0 + 8u * (B1 + 3 + x); };
+    auto BAR_PV = [&](int x) { return bar0 + 8u * (B1 + 5 + x); };
+    auto BAR_MF = [&](int k) { return bar0 + 8u * (B1 + 7 + k); };
+    auto BAR_ME = [&](int k) { return bar0 + 8u * (B1 + 7 + kMaskSlots + k); };
     uint32_t* maskbuf = (uint32_t*)(smem + C::OFF_MASK);
+    float2* stat = (float2*)(smem + C::OFF_STAT);
 
     uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
     volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
@@ -525,19 +528,23 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const Ctl ctl{abort_flag, P.status};
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < C::STAGES_K; ++s) {
             mbar_init(BAR_KF(s), 1);
-            mbar_init(BAR_VF(s), 1);
             mbar_init(BAR_KE(s), 1);
         }
-        mbar_init(BAR_SF(0), 1);
-        mbar_init(BAR_SF(1), 1);
-        mbar_init(BAR_PF, kSoftmaxWarps);
-        mbar_init(BAR_PV, 1);
-        mbar_init(BAR_QR, kSoftmaxWarps);
+        for (int s = 0; s < C::STAGES_V; ++s) {
+            mbar_init(BAR_VF(s), 1);
+            mbar_init(BAR_VE(s), 1);
+        }
+        mbar_init(BAR_QF, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR_SF(x), 1);
+            mbar_init(BAR_PF(x), 4);                    // the four warps of softmax warpgroup x
+            mbar_init(BAR_PV(x), 1);
+        }
         for (int k = 0; k < kMaskSlots; ++k) {
             mbar_init(BAR_MF(k), 2);
-            mbar_init(BAR_ME(k), kSoftmaxWarps);
+            mbar_init(BAR_ME(k), 4);                    // the warpgroup that consumed the slot
         }
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -556,75 +563,86 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t tmem = *tmem_slot;
 
     if (warp == kProducerWarp) {
-        // ---------------- TMA producer ----------------
-        if (lane == 0) {
+        // ---------------- TMA producer: lane 0 Q and K, lane 1 V ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+        if (lane == 0 && cnt > 0) {
+            mbar_expect_tx(BAR_QF, C::Q_BYTES);
+            for (int c = 0; c < D / 64; ++c)
+                tma_load_2d(s_base + C::OFF_Q + c * kRows * 128, &P.tm_q, c * 64, (int)row0, BAR_QF);
             for (int j = 0; j < cnt; ++j) {
-                const int st = j % C::STAGES;
-                const uint32_t use = (uint32_t)(j / C::STAGES);
-                if (j >= C::STAGES && !mbar_wait(BAR_KE(st), (use - 1) & 1, ctl)) break;
-                const int kv = VSA_ENTRY_KV(__ldg(entries + j));
-                const int krow = (int)(base_row + (long long)kv * BK);
+                const int st = j % C::STAGES_K;
+                if (j >= C::STAGES_K && !mbar_wait(BAR_KE(st), (uint32_t)(j / C::STAGES_K - 1) & 1, ctl)) break;
+                const int krow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
                 mbar_expect_tx(BAR_KF(st), C::KV_BYTES);
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_2d(s_base + C::OFF_K + st * C::KV_BYTES + c * BK * 128, &P.tm_k, c * 64, krow,
                                 BAR_KF(st));
+            }
+        } else if (lane == 1 && cnt > 0) {
+            for (int j = 0; j < cnt; ++j) {
+                const int st = j % C::STAGES_V;
+                if (j >= C::STAGES_V && !mbar_wait(BAR_VE(st), (uint32_t)(j / C::STAGES_V - 1) & 1, ctl)) break;
+                const int vrow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
                 mbar_expect_tx(BAR_VF(st), C::KV_BYTES);
                 for (int c = 0; c < D / 64; ++c)
-                    tma_load_2d(s_base + C::OFF_V + st * C::KV_BYTES + c * BK * 128, &P.tm_v, c * 64, krow,
+                    tma_load_2d(s_base + C::OFF_V + st * C::KV_BYTES + c * BK * 128, &P.tm_v, c * 64, vrow,
                                 BAR_VF(st));
             }
         }
+        __syncwarp();
     } else if (warp == kMmaWarp) {
         // ---------------- MMA issuer ----------------
-        // The whole warp runs this role so that the descriptor and address
-        // arithmetic stays warp-uniform; one elected lane issues each
-        // tcgen05.mma and tcgen05.commit.
-        // Order: QK_0, QK_1, PV_0, QK_2, PV_1, ...; QK_{j+2} reuses S_{j%2},
-        // which the softmax finished reading before it signalled P_j.
         // Descriptors are built once; per MMA only a compile-time offset is
         // added (the start-address field sits in the low bits and never carries).
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
         const uint32_t leader = elect_one();
-        if (cnt > 0 && mbar_wait_warp(BAR_QR, 0, ctl)) {
+        if (cnt > 0 && mbar_wait_warp(BAR_QF, 0, ctl)) {
+            tc_fence_after();
+            const uint64_t qdesc = smem_desc(s_base + C::OFF_Q, 16, 1024);
             const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
             const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
             constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
-            const uint32_t aQ = tmem + C::COL_Q;
-            const uint32_t aP = tmem + C::COL_P;
-            const uint32_t dO = tmem + C::COL_O;
-            tc_fence_after();
-            for (int j = 0; j <= cnt; ++j) {
-                if (j < cnt) {
-                    const int st = j % C::STAGES, b = j & 1;
-                    if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES) & 1, ctl)) break;
-                    tc_fence_after();
-                    const uint32_t dS = tmem + (b ? C::COL_S1 : C::COL_S0);
-                    const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
-                    mma_ts_lead<0>(dS, aQ, kd, C::IDESC_QK, leader);
+            // S_j = Q K_j^T into S_{j mod 2}; K_j's stage is released when it completes
+            auto issue_qk = [&](int j) -> bool {
+                const int st = j % C::STAGES_K;
+                if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES_K) & 1, ctl)) return false;
+                tc_fence_after();
+                const uint32_t dS = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
+                const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
+                mma_ss_lead<0>(dS, qdesc, kd, C::IDESC_QK, leader);
 #pragma unroll
-                    for (int kk = 1; kk < D / 16; ++kk)
-                        mma_ts_lead<1>(dS, aQ + kk * 8,
-                                       kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
-                                       C::IDESC_QK, leader);
-                    tc_commit_lead(BAR_SF(b), leader);
-                }
-                if (j >= 1) {
-                    const int jp = j - 1, stp = jp % C::STAGES;
-                    if (!mbar_wait_warp(BAR_PF, (uint32_t)jp & 1, ctl)) break;
-                    if (!mbar_wait_warp(BAR_VF(stp), (uint32_t)(jp / C::STAGES) & 1, ctl)) break;
-                    tc_fence_after();
-                    const uint64_t vd = vdesc0 + (uint64_t)stp * kStageStep;
-                    if (jp == 0) mma_ts_lead<0>(dO, aP, vd, C::IDESC_PV, leader);
-                    else mma_ts_lead<1>(dO, aP, vd, C::IDESC_PV, leader);
+                for (int kk = 1; kk < D / 16; ++kk)
+                    mma_ss_lead<1>(dS, qdesc + (uint64_t)((((kk >> 2) * (kRows * 128)) + (kk & 3) * 32) >> 4),
+                                   kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4), C::IDESC_QK,
+                                   leader);
+                tc_commit_lead(BAR_SF(j & 1), leader);
+                tc_commit_lead(BAR_KE(st), leader);
+                return true;
+            };
+            bool go = issue_qk(0) && (cnt < 2 || issue_qk(1));
+            for (int j = 0; go && j < cnt; ++j) {
+                const int x = j & 1, vs = j % C::STAGES_V;
+                if (!mbar_wait_warp(BAR_PF(x), (uint32_t)(j >> 1) & 1, ctl)) break;
+                if (!mbar_wait_warp(BAR_VF(vs), (uint32_t)(j / C::STAGES_V) & 1, ctl)) break;
+                tc_fence_after();
+                // O_x (+)= P_j V_j, P_j in the first BK/2 columns of S_x
+                const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
+                const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
+                const uint64_t vd = vdesc0 + (uint64_t)vs * kStageStep;
+                if (j < 2) mma_ts_lead<0>(dO, aP, vd, C::IDESC_PV, leader);
+                else mma_ts_lead<1>(dO, aP, vd, C::IDESC_PV, leader);
 #pragma unroll
-                    for (int kk = 1; kk < BK / 16; ++kk)
-                        mma_ts_lead<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
-                    tc_commit_lead(BAR_PV, leader);
-                    tc_commit_lead(BAR_KE(stp), leader);
-                }
+                for (int kk = 1; kk < BK / 16; ++kk)
+                    mma_ts_lead<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
+                tc_commit_lead(BAR_PV(x), leader);
+                tc_commit_lead(BAR_VE(vs), leader);
+                // S_{j+2} reuses S_x: queued behind PV_j, so P_j is read first
+                if (j + 2 < cnt) go = issue_qk(j + 2);
             }
         }
     } else if (warp >= kMaskWarp0) {
         // ---------------- mask workers (warps 10, 11) ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
         const int t = threadIdx.x - kMaskWarp0 * 32;      // rows t and t + 64
         const vsa_mask_spec m = P.specs[head];
         const vsa_row_ctx q0 = vsa_row_init(d, m, (long long)e * kRows + t);
@@ -657,99 +675,82 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             break;
         }
     } else {
-        // ---------------- softmax warps 0..7 ----------------
-        // lanes i and i + 16 share query row (TMEM lane) rbase + i; hc picks
-        // the column half of S, P and O, and the keep-bit words, they hold.
-        const int rbase = 32 * (warp & 3) + 16 * (warp >> 2);
-        const int row = rbase + (lane & 15);
-        const int hc = lane >> 4;
+        // ---------------- softmax warpgroups (warps 0..3: X = 0, 4..7: X = 1) ----------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+        const int X = warp >> 2;                          // list entries j with j mod 2 = X
+        const int row = threadIdx.x & (kRows - 1);        // TMEM lane
         const int half = row >> 6;                        // 64-row q tile of the row (warp-uniform)
-        const uint32_t lane_off = (uint32_t)rbase << 16;
-        const uint32_t tO = tmem + lane_off + C::COL_O;
-        const uint32_t tP = tmem + lane_off + C::COL_P;
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + (X ? C::COL_S1 : C::COL_S0);
+        const uint32_t tO = tmem + lane_off + (X ? C::COL_O1 : C::COL_O0);
         const vsa_mask_spec m = P.specs[head];
-
-        // Q row -> TMEM (the QK operand), two bf16 per column; each lane of
-        // the pair copies its half of the row
-        if (cnt > 0) {
-            const uint4* qrow = reinterpret_cast<const uint4*>(P.q + (row0 + row) * D + hc * (D / 2));
-            uint32_t qv[D / 4];
-#pragma unroll
-            for (int i = 0; i < D / 16; ++i) {
-                const uint4 x = __ldg(qrow + i);
-                qv[4 * i] = x.x; qv[4 * i + 1] = x.y; qv[4 * i + 2] = x.z; qv[4 * i + 3] = x.w;
-            }
-            tmem_st_half<D / 2>(tmem + lane_off + C::COL_Q, qv);
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR_QR);
-        }
         if (m.kind == VSA_MASK_STRIPE)
             for (int i = threadIdx.x; i < P.tab_words_t; i += 32 * kSoftmaxWarps)
                 ttab[i] = vsa_stripe_tword(m, d.T, i);
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
 
-        constexpr int NS = BK / 2;                        // S columns per lane
-        float m_run = -INFINITY;  // running max of scale*log2(e)*s (same in both lanes of the pair)
-        float l_run = 0.0f;       // partial row sum over this lane's columns
+        float m_run = -INFINITY;  // running max of scale*log2(e)*s over this warpgroup's tiles
+        float l_run = 0.0f;
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
         int ent_next = cnt > 0 ? __ldg(entries) : 0;
-        int kb = 0;                                       // boundary tiles seen so far
+        int kb = 0;                                       // boundary tiles of the list so far
         for (int j = 0; j < cnt && ok; ++j) {
-            const int b = j & 1;
             const int ent = ent_next;
             if (j + 1 < cnt) ent_next = __ldg(entries + j + 1);
+            const bool bnd = VSA_ENTRY_CLS(ent, 0) == VSA_TILE_BOUNDARY || VSA_ENTRY_CLS(ent, 1) == VSA_TILE_BOUNDARY;
+            if ((j & 1) != X) {                           // the other warpgroup's tile
+                kb += bnd ? 1 : 0;
+                continue;
+            }
             const int cls = VSA_ENTRY_CLS(ent, half);
-            const uint32_t tS = tmem + lane_off + (b ? C::COL_S1 : C::COL_S0);
-            if (!mbar_wait_warp(BAR_SF(b), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
-            float s[NS];
+            float s[BK];
             {
-                uint32_t sr[NS];
-                tmem_ld_half<BK>(tS, sr);
+                uint32_t sr[BK];
+#pragma unroll
+                for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
                 tmem_ld_wait();
 #pragma unroll
-                for (int c = 0; c < NS; ++c) {
+                for (int c = 0; c < BK; ++c) {
                     reg_fence(sr[c]);
                     s[c] = __uint_as_float(sr[c]);
                 }
             }
 
-            if (VSA_ENTRY_CLS(ent, 0) == VSA_TILE_BOUNDARY || VSA_ENTRY_CLS(ent, 1) == VSA_TILE_BOUNDARY) {
+            if (bnd) {
                 // keep bits from the mask workers; the slot is released after reading
                 const int slot = kb % kMaskSlots;
                 if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }
-                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + hc * (NS / 32) * kRows + row;
-                uint32_t mw[NS / 32];
+                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + row;
+                uint32_t mw[BK / 32];
 #pragma unroll
-                for (int wi = 0; wi < NS / 32; ++wi) mw[wi] = src[wi * kRows];
+                for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = src[wi * kRows];
                 __syncwarp();
                 if (lane == 0) mbar_arrive(BAR_ME(slot));
                 ++kb;
                 if (cls == VSA_TILE_BOUNDARY) {
 #pragma unroll
-                    for (int wi = 0; wi < NS / 32; ++wi)
+                    for (int wi = 0; wi < BK / 32; ++wi)
 #pragma unroll
                         for (int c = 0; c < 32; ++c)
                             if (!((mw[wi] >> c) & 1u)) s[wi * 32 + c] = -INFINITY;
                 }
             }
 
-            uint32_t pk[NS / 2];
+            uint32_t pk[BK / 2];
             bool need_o = false;
             float alpha = 1.0f;
             if (cls == VSA_TILE_EMPTY) {
 #pragma unroll
-                for (int c = 0; c < NS / 2; ++c) pk[c] = 0u;
+                for (int c = 0; c < BK / 2; ++c) pk[c] = 0u;
             } else {
-                // row max: independent chains of 3-input max over 32 columns
-                // each, then the other half of the row from the partner lane
-                float mc[NS / 32];
+                // row max: independent chains of 3-input max over 32 columns each
+                float mc[BK / 32];
 #pragma unroll
-                for (int g = 0; g < NS / 32; ++g) {
+                for (int g = 0; g < BK / 32; ++g) {
                     float a = s[g * 32];
 #pragma unroll
                     for (int c = 1; c < 31; c += 2) a = max3(a, s[g * 32 + c], s[g * 32 + c + 1]);
@@ -757,12 +758,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
                 float mx = mc[0];
 #pragma unroll
-                for (int g = 1; g < NS / 32; ++g) mx = fmaxf(mx, mc[g]);
-                mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+                for (int g = 1; g < BK / 32; ++g) mx = fmaxf(mx, mc[g]);
                 const float mxs = mx * sl;
                 if (mx != -INFINITY) {
                     if (m_run == -INFINITY) {
-                        m_run = mxs;  // nothing accumulated for this row yet: O row is 0
+                        m_run = mxs;  // nothing accumulated for this row yet: O_X row is 0
                     } else if (mxs > m_run + kRescaleThreshold) {
                         alpha = ex2(m_run - mxs);
                         l_run *= alpha;
@@ -774,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const unsigned long long mneg2 = f2_pack(mneg, mneg);
                 unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int i = 0; i < NS / 2; ++i) {
+                for (int i = 0; i < BK / 2; ++i) {
                     float x0, x1;
                     f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2, mneg2), x0, x1);
                     const float p0 = ex2(x0);
@@ -789,55 +789,78 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 f2_unpack(acc[3], a6, a7);
                 l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
             }
-            // PV_{j-1} must be complete before P is overwritten and before O is
-            // rescaled; every phase of its barrier is awaited in order
-            if (j > 0) {
-                if (!mbar_wait_warp(BAR_PV, (uint32_t)(j - 1) & 1, ctl)) { ok = false; break; }
-                tc_fence_after();
-            }
+            // S_j complete implies PV_{j-2}, the last MMA into O_X, is complete
+            // (one thread's MMAs run in order), so O_X can be rescaled here
             if (__any_sync(0xFFFFFFFFu, need_o)) {
 #pragma unroll
-                for (int c = 0; c < D / 64; ++c) {
+                for (int c = 0; c < D / 32; ++c) {
                     uint32_t ov[32];
-                    tmem_ld_pair32<D / 2>(tO + c * 32, ov);
+                    tmem_ld32(tO + c * 32, ov);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
                         reg_fence(ov[i]);
                         ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
                     }
-                    tmem_st_pair32<D / 2>(tO + c * 32, ov);
+                    tmem_st32(tO + c * 32, ov);
                 }
             }
-            tmem_st_half<BK / 2>(tP, pk);
+            // P_j (bf16 pairs) over the first BK/2 columns of S_X
+#pragma unroll
+            for (int c = 0; c < BK / 64; ++c) tmem_st32(tS + c * 32, pk + c * 32);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR_PF);
+            if (lane == 0) mbar_arrive(BAR_PF(X));
         }
 
-        // ---------------- epilogue ----------------
+        // ---------------- epilogue: merge the two warpgroups' partial softmaxes ----------------
+        // Warpgroup 0 had (cnt + 1) / 2 tiles, warpgroup 1 cnt / 2.  Each waits
+        // for the last PV into its own accumulator (its barrier is at most one
+        // phase behind, so the parity wait is exact), then the named barrier
+        // hands both results to both warpgroups.
+        const int n0 = (cnt + 1) >> 1, n1 = cnt >> 1;
+        const int nx = X ? n1 : n0;
+        bool have_o = ok;
+        if (have_o && nx > 0) have_o = mbar_wait_warp(BAR_PV(X), (uint32_t)(nx - 1) & 1, ctl);
+        stat[X * kRows + row] = make_float2(m_run, l_run);
+        tc_fence_before();
+        asm volatile("bar.sync 2, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        tc_fence_after();
+        have_o = have_o && !*abort_flag;
+        const float2 st0 = stat[row], st1 = stat[kRows + row];
+        const float mm = fmaxf(st0.x, st1.x);
+        const float w0 = st0.y > 0.0f ? ex2(st0.x - mm) : 0.0f;
+        const float w1 = st1.y > 0.0f ? ex2(st1.x - mm) : 0.0f;
+        const float l_row = w0 * st0.y + w1 * st1.y;
+        const float inv = l_row > 0.0f ? 1.0f / l_row : 0.0f;
         const long long orow = row0 + row;
-        bool have_o = ok && cnt > 0;
-        if (have_o) {
-            have_o = mbar_wait_warp(BAR_PV, (uint32_t)(cnt - 1) & 1, ctl);
-            tc_fence_after();
-        }
-        const float l_row = l_run + __shfl_xor_sync(0xFFFFFFFFu, l_run, 16);
-        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D + hc * (D / 2));
-        if (have_o) {
-            const float inv = l_row > 0.0f ? 1.0f / l_row : 0.0f;
+        // warpgroup X writes columns [X D/2, (X+1) D/2) of the output row
+        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D + X * (D / 2));
+        if (have_o && cnt > 0) {
 #pragma unroll
             for (int c = 0; c < D / 64; ++c) {
-                uint32_t ov[32];
-                tmem_ld_pair32<D / 2>(tO + c * 32, ov);
+                const int col = X * (D / 2) + c * 32;
+                uint32_t o0[32], o1[32];
+                tmem_ld32(tmem + lane_off + C::COL_O0 + col, o0);
+                if (n1 > 0) tmem_ld32(tmem + lane_off + C::COL_O1 + col, o1);
                 tmem_ld_wait();
                 uint32_t pkd[16];
 #pragma unroll
                 for (int i = 0; i < 32; i += 2) {
-                    reg_fence(ov[i]);
-                    reg_fence(ov[i + 1]);
-                    pkd[i >> 1] = pack_bf16(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                    float v[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        reg_fence(o0[i + h]);
+                        const float x0 = w0 > 0.0f ? __uint_as_float(o0[i + h]) * w0 : 0.0f;
+                        float x1 = 0.0f;
+                        if (n1 > 0) {
+                            reg_fence(o1[i + h]);
+                            x1 = w1 > 0.0f ? __uint_as_float(o1[i + h]) * w1 : 0.0f;
+                        }
+                        v[h] = (x0 + x1) * inv;
+                    }
+                    pkd[i >> 1] = pack_bf16(v[0], v[1]);
                 }
 #pragma unroll
                 for (int i = 0; i < 4; ++i)
@@ -847,8 +870,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
 #pragma unroll
             for (int i = 0; i < D / 16; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
         }
-        if (hc == 0)
-            P.lse[orow] = (l_row > 0.0f) ? (m_run + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
+        if (X == 0) P.lse[orow] = (l_row > 0.0f) ? (mm + __log2f(l_row)) * 0.69314718055994531f : -INFINITY;
     }
 
     // ---------------- teardown ----------------
@@ -927,8 +949,9 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
 
     AttnParams P;
     memset(&P, 0, sizeof P);
-    if (!make_map(&P.tm_k, k, rows, D, d.Bk) || !make_map(&P.tm_v, v, rows, D, d.Bk)) return VSA_ERR_CUDA;
-    P.q = (const __nv_bfloat16*)q;
+    if (!make_map(&P.tm_q, q, rows, D, kRows) || !make_map(&P.tm_k, k, rows, D, d.Bk) ||
+        !make_map(&P.tm_v, v, rows, D, d.Bk))
+        return VSA_ERR_CUDA;
     P.o = (__nv_bfloat16*)o;
     P.lse = lse;
     P.list_cnt = plan->d_list_cnt;
