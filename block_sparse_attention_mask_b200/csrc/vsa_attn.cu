@@ -68,6 +68,7 @@ constexpr int kRegsLaunch = 168;
 constexpr int kMaskSlots = 4;                     // boundary-tile masks in flight
 constexpr int kRows = VSA_EXEC_ROWS;              // 128 query rows per CTA
 constexpr long long kWatchdogCycles = 1LL << 31;  // ~1 s at 2 GHz per wait
+constexpr long long kDrainCycles = 1LL << 24;     // ~8 ms for a role's own copies or MMAs
 constexpr float kRescaleThreshold = 8.0f;         // log2 units
 
 template <int D, int BK>
@@ -102,10 +103,12 @@ struct Cfg {
     static constexpr int OFF_STAT = OFF_MASK + kMaskSlots * MASK_SLOT_WORDS * 4;
     static constexpr int OFF_BAR = OFF_STAT + 2 * kRows * 8;
     // barriers: k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], q_full,
-    //           s_full[2], p_full[2], pv_done[2], mask_full[M], mask_empty[M]
-    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 7 + 2 * kMaskSlots;
-    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;      // tmem addr (4) + abort (4)
-    static constexpr int OFF_TAB = (OFF_MISC + 8 + 15) / 16 * 16;
+    //           s_full[2], p_full[2], pv_done[2], mask_full[M], mask_empty[M], mma_drain
+    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 8 + 2 * kMaskSlots;
+    // tmem addr, abort flag, and for the teardown after an abort: K and V
+    // copies started, MMAs started (4 bytes each)
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_TAB = (OFF_MISC + 20 + 15) / 16 * 16;
     // instruction descriptors (kind::f16): D fp32, A and B bf16
     //   bits [4,6) D format = 1 (f32); [7,10) A = 1 (bf16); [10,13) B = 1 (bf16);
     //   bit 15 A major (0 = K); bit 16 B major (1 = MN); [17,23) N >> 3; [24,29) M >> 4
@@ -185,6 +188,16 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, c
             *c.abort = 1;
             return false;
         }
+    }
+}
+
+// Wait, ignoring the abort flag, for a role's own copies or MMAs still in
+// flight before the CTA frees TMEM and exits; gives up after `limit` cycles.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, long long limit)
+{
+    if (mbar_try_wait(bar, parity)) return;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity) && clock64() - t0 <= limit) {
     }
 }
 
@@ -518,11 +531,15 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     auto BAR_PV = [&](int x) { return bar0 + 8u * (B1 + 5 + x); };
     auto BAR_MF = [&](int k) { return bar0 + 8u * (B1 + 7 + k); };
     auto BAR_ME = [&](int k) { return bar0 + 8u * (B1 + 7 + kMaskSlots + k); };
+    const uint32_t BAR_DR = bar0 + 8u * (B1 + 7 + 2 * kMaskSlots);
     uint32_t* maskbuf = (uint32_t*)(smem + C::OFF_MASK);
     float2* stat = (float2*)(smem + C::OFF_STAT);
 
     uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
     volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
+    // for the teardown after an abort, kept in shared memory rather than in
+    // registers live across every role: [K copies, V copies, MMAs] started
+    volatile int* issued = (volatile int*)(smem + C::OFF_MISC + 8);
     uint32_t* stab = (uint32_t*)(smem + C::OFF_TAB);
     uint32_t* ttab = stab + P.tab_words_s;
     const Ctl ctl{abort_flag, P.status};
@@ -537,6 +554,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             mbar_init(BAR_VE(s), 1);
         }
         mbar_init(BAR_QF, 1);
+        mbar_init(BAR_DR, 1);
         for (int x = 0; x < 2; ++x) {
             mbar_init(BAR_SF(x), 1);
             mbar_init(BAR_PF(x), 4);                    // the four warps of softmax warpgroup x
@@ -547,6 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             mbar_init(BAR_ME(k), 4);                    // the warpgroup that consumed the slot
         }
         *abort_flag = 0;
+        issued[0] = issued[1] = issued[2] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
@@ -569,7 +588,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             mbar_expect_tx(BAR_QF, C::Q_BYTES);
             for (int c = 0; c < D / 64; ++c)
                 tma_load_2d(s_base + C::OFF_Q + c * kRows * 128, &P.tm_q, c * 64, (int)row0, BAR_QF);
-            for (int j = 0; j < cnt; ++j) {
+            int nk = 0;
+            for (int j = 0; j < cnt; ++j, nk = j) {
                 const int st = j % C::STAGES_K;
                 if (j >= C::STAGES_K && !mbar_wait(BAR_KE(st), (uint32_t)(j / C::STAGES_K - 1) & 1, ctl)) break;
                 const int krow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
@@ -578,8 +598,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     tma_load_2d(s_base + C::OFF_K + st * C::KV_BYTES + c * BK * 128, &P.tm_k, c * 64, krow,
                                 BAR_KF(st));
             }
+            issued[0] = nk;
         } else if (lane == 1 && cnt > 0) {
-            for (int j = 0; j < cnt; ++j) {
+            int nv = 0;
+            for (int j = 0; j < cnt; ++j, nv = j) {
                 const int st = j % C::STAGES_V;
                 if (j >= C::STAGES_V && !mbar_wait(BAR_VE(st), (uint32_t)(j / C::STAGES_V - 1) & 1, ctl)) break;
                 const int vrow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
@@ -588,6 +610,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     tma_load_2d(s_base + C::OFF_V + st * C::KV_BYTES + c * BK * 128, &P.tm_v, c * 64, vrow,
                                 BAR_VF(st));
             }
+            issued[1] = nv;
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
@@ -619,7 +642,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tc_commit_lead(BAR_KE(st), leader);
                 return true;
             };
-            bool go = issue_qk(0) && (cnt < 2 || issue_qk(1));
+            bool go = issue_qk(0);
+            if (go && leader) issued[2] = 1;
+            go = go && (cnt < 2 || issue_qk(1));
             for (int j = 0; go && j < cnt; ++j) {
                 const int x = j & 1, vs = j % C::STAGES_V;
                 if (!mbar_wait_warp(BAR_PF(x), (uint32_t)(j >> 1) & 1, ctl)) break;
@@ -876,6 +901,30 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     // ---------------- teardown ----------------
     tc_fence_before();
     __syncthreads();
+    if (*abort_flag) {
+        // After a watchdog abort some copies or MMAs may still be in flight:
+        // each role waits (bounded) for its own before TMEM is freed.  A
+        // normal run consumed all of them already.
+        if (warp == kProducerWarp && lane == 0 && cnt > 0) {
+            const int nk = issued[0];
+            mbar_drain(BAR_QF, 0, kDrainCycles);
+            for (int j = nk > C::STAGES_K ? nk - C::STAGES_K : 0; j < nk; ++j)
+                mbar_drain(BAR_KF(j % C::STAGES_K), (uint32_t)(j / C::STAGES_K) & 1, kDrainCycles);
+        }
+        if (warp == kProducerWarp && lane == 1) {
+            const int nv = issued[1];
+            for (int j = nv > C::STAGES_V ? nv - C::STAGES_V : 0; j < nv; ++j)
+                mbar_drain(BAR_VF(j % C::STAGES_V), (uint32_t)(j / C::STAGES_V) & 1, kDrainCycles);
+        }
+        if (warp == kMmaWarp && issued[2]) {
+            const uint32_t leader = elect_one();
+            tc_commit_lead(BAR_DR, leader);
+            if (leader) mbar_drain(BAR_DR, 0, kDrainCycles);
+            __syncwarp();
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
     if (warp == kMmaWarp) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
