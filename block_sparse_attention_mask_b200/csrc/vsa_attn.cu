@@ -101,7 +101,9 @@ struct Cfg {
     static constexpr int MASK_SLOT_WORDS = (BK / 32) * kRows;
     // per-warpgroup row statistics (running max, running sum) for the merge
     static constexpr int OFF_STAT = OFF_MASK + kMaskSlots * MASK_SLOT_WORDS * 4;
-    static constexpr int OFF_BAR = OFF_STAT + 2 * kRows * 8;
+    // per-row mask context (query coordinates, STA window), read on boundary tiles
+    static constexpr int OFF_ROWCTX = OFF_STAT + 2 * kRows * 8;
+    static constexpr int OFF_BAR = OFF_ROWCTX + kRows * (int)sizeof(vsa_row_ctx);
     // barriers: k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], q_full,
     //           s_full[2], p_full[2], pv_done[2], mask_full[M], mask_empty[M], mma_drain
     static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 8 + 2 * kMaskSlots;
@@ -359,12 +361,119 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
            ((uint64_t)((sbo >> 4) & 0x3FFF) << 32) | (1ull << 46) | (2ull << 61);
 }
 
-// Mask-worker loop, specialised on the mask kind (uniform per CTA) so that
-// no per-run branch on the kind remains.  Thread t of the two mask warps
-// writes the keep bits of rows t and t + 64 for every boundary tile of the
-// list into slot (k mod kMaskSlots) of the ring, k = boundary tiles so far.
-// The run descriptors of a tile (bw keys sharing t and h each) are loaded
-// once per warp, one per lane, and broadcast with warp shuffles.
+// Keep bits of query row q for a kv tile that is one box inside a unit
+// (box_nh > 0): run r of the tile (bw keys sharing t and h) sits at
+// (t0 + r / box_nh, h0 + r mod box_nh) with the same first column w0 and the
+// same number of real keys for every run, so a run costs a few operations.
+// v is the tile's first run descriptor; bit c of words[c / 32] is key c.
+template <int KIND, int BK>
+__device__ __forceinline__ void box_row_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                             const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
+                                             uint32_t (&words)[BK / 32])
+{
+    const int t0 = v.x & 0xFFFF, h0 = v.x >> 16, w0 = v.y & 0xFFFF;
+    const int bw = d.bw;
+    const int wv = tile_real ? max(0, min(bw, d.W - w0)) : 0;
+    const uint32_t vm = vsa_low_bits(wv);
+    // row-invariant parts for this tile
+    uint32_t wmask = 0;             // temporal: kept w offsets of a run
+    bool sta_in = false;            // STA: the tile's unit is in the row's window
+    if (KIND == VSA_MASK_SVG_TEMPORAL) {
+        const int lo = max(q.wq - m.rw, w0) - w0;
+        const int hi = min(q.wq + m.rw, w0 + wv - 1) - w0;
+        wmask = (lo <= hi) ? (vsa_low_bits(hi - lo + 1) << lo) : 0u;
+    }
+    if (KIND == VSA_MASK_STA) {
+        const int ut = t0 / d.bt, uh = h0 / d.bh, uw = w0 / d.bw;
+        sta_in = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h && uh < q.sta_h + q.kk_h &&
+                 uw >= q.sta_w && uw < q.sta_w + q.kk_w;
+    }
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) words[wi] = 0u;
+    uint32_t acc = 0;
+    int tt = t0, dh = 0;
+    bool tvalid = false, sinkhit = false, tkeep = true;
+    int xbase = 0;
+    for (int r = 0; r < d.nseg; ++r) {
+        if (dh == 0) {              // a new t-slice of the tile: everything but h is fixed
+            tvalid = q.real && tt < d.T;
+            sinkhit = m.sink && tt == 0;
+            tkeep = true;
+            if (KIND == VSA_MASK_SVG_SPATIAL) tkeep = vsa_iabs(tt - q.tq) <= m.rt;
+            if (KIND == VSA_MASK_STRIPE) {
+                const int it = tt - q.tq + d.T - 1;
+                tkeep = tvalid && ((ttab[it >> 5] >> (it & 31)) & 1u);
+            }
+            xbase = h0 * d.W + w0 - q.sq + d.H * d.W - 1;
+        }
+        const int hh = h0 + dh;
+        uint32_t b = 0;
+        if (KIND == VSA_MASK_STRIPE) {
+            const int x = xbase + dh * d.W;
+            const uint32_t win = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31) & vm;
+            b = tkeep ? win : 0u;
+        } else if (KIND == VSA_MASK_SVG_TEMPORAL) {
+            b = vsa_iabs(hh - q.hq) <= m.rh ? wmask : 0u;
+        } else if (KIND == VSA_MASK_SVG_SPATIAL) {
+            b = tkeep ? vm : 0u;
+        } else if (KIND == VSA_MASK_STA) {
+            b = sta_in ? vm : 0u;
+        } else {
+            b = vm;
+        }
+        if (sinkhit) b = vm;
+        if (!(tvalid && hh < d.H)) b = 0u;
+        const int col = r * bw;
+        acc |= b << (col & 31);
+        if (((col + bw) & 31) == 0) {          // last run of a 32-key word (bw divides 32)
+#pragma unroll
+            for (int wi = 0; wi < BK / 32; ++wi) words[wi] = (col >> 5) == wi ? acc : words[wi];
+            acc = 0;
+        }
+        if (++dh == d.box_nh) {
+            dh = 0;
+            ++tt;
+        }
+    }
+}
+
+template <int BK>
+__device__ __forceinline__ void box_row_bits_any(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                                 const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
+                                                 uint32_t (&words)[BK / 32])
+{
+    vsa_mask_spec mk = m;
+    switch (m.kind) {
+    case VSA_MASK_FULL:
+        mk.kind = VSA_MASK_FULL;
+        box_row_bits<VSA_MASK_FULL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
+        break;
+    case VSA_MASK_SVG_SPATIAL:
+        mk.kind = VSA_MASK_SVG_SPATIAL;
+        box_row_bits<VSA_MASK_SVG_SPATIAL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
+        break;
+    case VSA_MASK_SVG_TEMPORAL:
+        mk.kind = VSA_MASK_SVG_TEMPORAL;
+        box_row_bits<VSA_MASK_SVG_TEMPORAL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
+        break;
+    case VSA_MASK_STA:
+        mk.kind = VSA_MASK_STA;
+        box_row_bits<VSA_MASK_STA, BK>(mk, d, q, stab, ttab, v, tile_real, words);
+        break;
+    default:
+        mk.kind = VSA_MASK_STRIPE;
+        box_row_bits<VSA_MASK_STRIPE, BK>(mk, d, q, stab, ttab, v, tile_real, words);
+        break;
+    }
+}
+
+// Mask-worker loop for kv tiles made of several boxes (box_nh = 0),
+// specialised on the mask kind (uniform per CTA) so that no per-run branch on
+// the kind remains.  Thread t of the two mask warps writes the keep bits of
+// rows t and t + 64 for every boundary tile of the list into slot
+// (k mod kMaskSlots) of the ring, k = boundary tiles so far.  The run
+// descriptors of a tile (bw keys sharing t and h each) are loaded once per
+// warp, one per lane, and broadcast with warp shuffles.
 template <int KIND, int BK>
 __device__ __forceinline__ void mask_worker_loop(const vsa_mask_spec& m_in, const vsa_dims& d,
                                                  const vsa_row_ctx& q0, const vsa_row_ctx& q1,
@@ -387,82 +496,6 @@ __device__ __forceinline__ void mask_worker_loop(const vsa_mask_spec& m_in, cons
         const int slot = kb % kMaskSlots;
         const int kv = VSA_ENTRY_KV(ent);
         const int2* sg = seg + (size_t)kv * nseg;
-        if (d.box_nh > 0) {
-            // The tile is one box inside a unit: run r sits at t0 + r / box_nh,
-            // h0 + r % box_nh, with the same first column w0 and width for every
-            // run, so each run needs only a few operations per row.
-            const int2 v = __ldg(sg);
-            const int t0 = v.x & 0xFFFF, h0 = v.x >> 16, w0 = v.y & 0xFFFF;
-            const bool tile_real = (long long)kv * BK < d.Npad;
-            const int wv = tile_real ? max(0, min(bw, d.W - w0)) : 0;
-            const uint32_t vm = vsa_low_bits(wv);
-            if (kb >= kMaskSlots &&
-                !mbar_wait_warp(bar_me0 + 8u * slot, (uint32_t)(kb / kMaskSlots - 1) & 1, ctl))
-                return;
-            uint32_t* dst = maskbuf + slot * MASK_SLOT_WORDS;
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-                const vsa_row_ctx& q = which ? q1 : q0;
-                const int row = t + which * 64;
-                // row-invariant parts for this tile
-                uint32_t wmask = 0;             // temporal: kept w offsets of the run
-                bool sta_in = false;            // STA: the tile's unit is in the row's window
-                if (KIND == VSA_MASK_SVG_TEMPORAL) {
-                    const int lo = max(q.wq - m.rw, w0) - w0;
-                    const int hi = min(q.wq + m.rw, w0 + wv - 1) - w0;
-                    wmask = (lo <= hi) ? (vsa_low_bits(hi - lo + 1) << lo) : 0u;
-                }
-                if (KIND == VSA_MASK_STA) {
-                    const int ut = t0 / d.bt, uh = h0 / d.bh, uw = w0 / d.bw;
-                    sta_in = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h &&
-                             uh < q.sta_h + q.kk_h && uw >= q.sta_w && uw < q.sta_w + q.kk_w;
-                }
-                uint32_t acc = 0;
-                for (int r0 = 0; r0 < nseg; r0 += d.box_nh) {
-                    // one t-slice of the tile: everything but h is fixed here
-                    const int tt = t0 + r0 / d.box_nh;
-                    const bool tvalid = q.real && tt < d.T;
-                    const bool sinkhit = m.sink && tt == 0;
-                    bool tkeep = true;
-                    if (KIND == VSA_MASK_SVG_SPATIAL) tkeep = vsa_iabs(tt - q.tq) <= m.rt;
-                    if (KIND == VSA_MASK_STRIPE) {
-                        const int it = tt - q.tq + d.T - 1;
-                        tkeep = tvalid && ((ttab[it >> 5] >> (it & 31)) & 1u);
-                    }
-                    const int xbase = h0 * d.W + w0 - q.sq + d.H * d.W - 1;
-#pragma unroll 8
-                    for (int dh = 0; dh < d.box_nh; ++dh) {
-                        const int hh = h0 + dh;
-                        uint32_t b = 0;
-                        if (KIND == VSA_MASK_STRIPE) {
-                            const int x = xbase + dh * d.W;
-                            const uint32_t win = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31) & vm;
-                            b = (tkeep ? win : 0u);
-                        } else if (KIND == VSA_MASK_SVG_TEMPORAL) {
-                            b = vsa_iabs(hh - q.hq) <= m.rh ? wmask : 0u;
-                        } else if (KIND == VSA_MASK_SVG_SPATIAL) {
-                            b = tkeep ? vm : 0u;
-                        } else if (KIND == VSA_MASK_STA) {
-                            b = sta_in ? vm : 0u;
-                        } else {
-                            b = vm;
-                        }
-                        if (sinkhit) b = vm;
-                        if (!(tvalid && hh < d.H)) b = 0u;
-                        const int col = (r0 + dh) * bw;
-                        acc |= b << (col & 31);
-                        if (((col + bw) & 31) == 0) {
-                            dst[(col >> 5) * kRows + row] = acc;
-                            acc = 0;
-                        }
-                    }
-                }
-            }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar_mf0 + 8u * slot);
-            ++kb;
-            continue;
-        }
         int2 rr[BK / 32];
 #pragma unroll
         for (int i = 0; i < BK / 32; ++i) rr[i] = (i * 32 + lane < nseg) ? __ldg(sg + i * 32 + lane) : make_int2(0, 0);
@@ -534,6 +567,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const uint32_t BAR_DR = bar0 + 8u * (B1 + 7 + 2 * kMaskSlots);
     uint32_t* maskbuf = (uint32_t*)(smem + C::OFF_MASK);
     float2* stat = (float2*)(smem + C::OFF_STAT);
+    vsa_row_ctx* rowctx = (vsa_row_ctx*)(smem + C::OFF_ROWCTX);
 
     uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
     volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
@@ -677,7 +711,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int i = t; i < P.tab_words_s; i += 64) stab[i] = src[i];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
-        switch (m.kind) {
+        // single-box tiles are evaluated by the softmax threads themselves
+        if (d.box_nh == 0) switch (m.kind) {
         case VSA_MASK_FULL:
             mask_worker_loop<VSA_MASK_FULL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane, maskbuf,
                                                 BAR_MF(0), BAR_ME(0), ctl);
@@ -712,8 +747,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (m.kind == VSA_MASK_STRIPE)
             for (int i = threadIdx.x; i < P.tab_words_t; i += 32 * kSoftmaxWarps)
                 ttab[i] = vsa_stripe_tword(m, d.T, i);
+        if (X == 0) rowctx[row] = vsa_row_init(d, m, (long long)e * kRows + row);
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
 
+        const bool box = d.box_nh > 0;                    // boundary bits computed here, not by mask workers
         float m_run = -INFINITY;  // running max of scale*log2(e)*s over this warpgroup's tiles
         float l_run = 0.0f;
         const float sl = P.scale_log2;
@@ -730,6 +767,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 continue;
             }
             const int cls = VSA_ENTRY_CLS(ent, half);
+            // keep bits of a single-box boundary tile, computed while S_j is in flight
+            uint32_t mw[BK / 32];
+            if (bnd && box) {
+                const int kv = VSA_ENTRY_KV(ent);
+                const vsa_row_ctx q = rowctx[row];
+                box_row_bits_any<BK>(m, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                                     (long long)kv * BK < d.Npad, mw);
+            }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
             float s[BK];
@@ -746,16 +791,17 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
 
             if (bnd) {
-                // keep bits from the mask workers; the slot is released after reading
-                const int slot = kb % kMaskSlots;
-                if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }
-                const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + row;
-                uint32_t mw[BK / 32];
+                if (!box) {
+                    // keep bits from the mask workers; the slot is released after reading
+                    const int slot = kb % kMaskSlots;
+                    if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }
+                    const uint32_t* src = maskbuf + slot * C::MASK_SLOT_WORDS + row;
 #pragma unroll
-                for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = src[wi * kRows];
-                __syncwarp();
-                if (lane == 0) mbar_arrive(BAR_ME(slot));
-                ++kb;
+                    for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = src[wi * kRows];
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR_ME(slot));
+                    ++kb;
+                }
                 if (cls == VSA_TILE_BOUNDARY) {
 #pragma unroll
                     for (int wi = 0; wi < BK / 32; ++wi)
