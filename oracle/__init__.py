@@ -29,7 +29,7 @@ _lib = None
 class _Mask(ctypes.Structure):
     _fields_ = [(k, ctypes.c_int32) for k in
                 ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-                 "Tw", "To", "Ts", "Sw", "So", "Ss")]
+                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")]
 
 
 class _Grid(ctypes.Structure):
@@ -56,6 +56,8 @@ def _load():
         lib.orc_padded_tokens.argtypes = [P(_Grid)]
         lib.orc_tile_major_order.restype = ctypes.c_int64
         lib.orc_tile_major_order.argtypes = [P(_Grid), ctypes.c_int64, ctypes.c_void_p]
+        lib.orc_frame0_first_order.restype = ctypes.c_int64
+        lib.orc_frame0_first_order.argtypes = [P(_Grid), ctypes.c_int64, ctypes.c_void_p]
         lib.orc_keep.restype = ctypes.c_int
         lib.orc_keep.argtypes = [P(_Mask), P(_Grid), ctypes.c_int64, ctypes.c_int64]
         lib.orc_keep_matrix.restype = ctypes.c_int
@@ -100,15 +102,17 @@ def padded_tokens(grid, unit) -> int:
     return int(_load().orc_padded_tokens(ctypes.byref(_grid(grid, unit))))
 
 
-def tile_major_order(grid, unit, n_slots: Optional[int] = None) -> np.ndarray:
-    """perm[slot] = natural token index or -1 (padding)."""
+def tile_major_order(grid, unit, n_slots: Optional[int] = None, layout: int = 0) -> np.ndarray:
+    """perm[slot] = natural token index or -1 (padding), for a head's layout:
+    0 tile-major over 3D units, 1 frame 0 first then position-major."""
     g = _grid(grid, unit)
     if n_slots is None:
         n_slots = padded_tokens(grid, unit)
     perm = np.empty(n_slots, dtype=np.int32)
-    r = _load().orc_tile_major_order(ctypes.byref(g), n_slots, perm.ctypes.data)
+    fn = _load().orc_frame0_first_order if layout == 1 else _load().orc_tile_major_order
+    r = fn(ctypes.byref(g), n_slots, perm.ctypes.data)
     if r < 0:
-        raise ValueError("n_slots smaller than the padded grid")
+        raise ValueError("n_slots smaller than the grid")
     return perm
 
 

@@ -16,6 +16,16 @@
  *    "Fast Video Generation with Sliding Tile Attention", section 3 (tokens of
  *    a tile numbered contiguously).  Padding slots map to -1.
  *
+ *  - orc_frame0_first_order: the layout for temporal heads ("Sparse VideoGen:
+ *    accelerating video diffusion attention on TPU", "arranging tokens for
+ *    efficient temporal access"; "Video diffusion long-sequence attention and
+ *    sparsity", section 7.2: tokens of one spatial position across frames made
+ *    contiguous, so a temporal head's diagonal stripe becomes contiguous
+ *    bands).  Reading: the frame-0 sink would otherwise put one kept key in
+ *    every tile, so frame 0 is listed first, in (h,w) row-major order, then
+ *    each (h,w) position in row-major order with its frames 1..T-1 in order.
+ *    No padding inside; slots past T*H*W map to -1.
+ *
  *  - orc_keep: the element predicate of each mask family on real coordinates.
  *      spatial / temporal heads + frame-0 sink: "Sparse VideoGen: accelerating
  *        video diffusion attention on TPU", section on SVG heads (figure 3);
@@ -31,7 +41,7 @@
  *    lse = log sum exp over kept keys.
  *
  *  - orc_tile_counts: for q tiles of Bq slots and kv tiles of Bk slots in
- *    tile-major order, the number of kept (real query, key slot) pairs, by
+ *    the head's order, the number of kept (real query, key slot) pairs, by
  *    brute force.  The three-class map (empty / boundary / full) is read off
  *    those counts ("Sparse VideoGen ... on TPU", section "logical sparsity is
  *    not physical sparsity").
@@ -46,6 +56,7 @@
 
 typedef struct {
     int32_t kind, sink, rt, rh, rw, kt, kh, kw, Tw, To, Ts, Sw, So, Ss;
+    int32_t layout;   /* token order of the head: 0 tile-major, 1 frame 0 first */
 } orc_mask;
 
 typedef struct {
@@ -86,6 +97,30 @@ int64_t orc_tile_major_order(const orc_grid* g, int64_t n_slots, int32_t* perm)
                         }
     while (slot < n_slots) perm[slot++] = -1;
     return npad;
+}
+
+/* perm[slot] = natural token index: frame 0 in (h,w) order, then every (h,w)
+   position with its frames 1..T-1.  Returns T*H*W, or -1 if n_slots is too
+   small. */
+int64_t orc_frame0_first_order(const orc_grid* g, int64_t n_slots, int32_t* perm)
+{
+    const int64_t n = (int64_t)g->T * g->H * g->W;
+    if (n_slots < n) return -1;
+    int64_t slot = 0;
+    for (int h = 0; h < g->H; ++h)
+        for (int w = 0; w < g->W; ++w) perm[slot++] = (int32_t)((int64_t)h * g->W + w);
+    for (int h = 0; h < g->H; ++h)
+        for (int w = 0; w < g->W; ++w)
+            for (int t = 1; t < g->T; ++t) perm[slot++] = (int32_t)(((int64_t)t * g->H + h) * g->W + w);
+    while (slot < n_slots) perm[slot++] = -1;
+    return n;
+}
+
+/* The order of a head, by its layout field. */
+static int64_t head_order(const orc_mask* m, const orc_grid* g, int64_t n_slots, int32_t* perm)
+{
+    if (m->layout == 1) return orc_frame0_first_order(g, n_slots, perm);
+    return orc_tile_major_order(g, n_slots, perm);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -319,7 +354,7 @@ int orc_tile_counts(const orc_mask* m, const orc_grid* g, int64_t n_slots, int B
     if (!m || !g || Bq <= 0 || Bk <= 0 || n_slots % Bq || n_slots % Bk) return -1;
     int32_t* perm = (int32_t*)malloc(sizeof(int32_t) * n_slots);
     if (!perm) return -2;
-    if (orc_tile_major_order(g, n_slots, perm) < 0) { free(perm); return -1; }
+    if (head_order(m, g, n_slots, perm) < 0) { free(perm); return -1; }
     for (int64_t i = 0; i < nqt; ++i)
         if (qtiles[i] < 0 || qtiles[i] >= n_slots / Bq) { free(perm); return -1; }
     int32_t* coords = (int32_t*)malloc(sizeof(int32_t) * 3 * n_slots);

@@ -343,3 +343,61 @@ def test_stripe_parameter_draw_is_in_range_and_seeded():
     for p in p1:
         assert 1 <= p["Tw"] <= 4 and 0 <= p["To"] <= 2 and p["Ts"] in (21, 7, 5)
         assert 80 <= p["Sw"] <= 720 and p["So"] in (0, 80, 160) and p["Ss"] in (3600, 1200, 400)
+
+
+# --- layout 1 (frame 0 first, then position-major) for temporal heads -------------
+
+
+def test_frame0_first_order_structure():
+    # "Sparse VideoGen ... on TPU", "arranging tokens for efficient temporal
+    # access": tokens of one spatial position across frames become contiguous;
+    # frame 0 (the sink) comes first.
+    T, H, Wd = 4, 3, 5
+    HW, N = H * Wd, T * H * Wd
+    perm = oracle.tile_major_order((T, H, Wd), (1, 1, 1), 128, layout=1)
+    assert sorted(perm[:N].tolist()) == list(range(N))          # a bijection onto the real tokens
+    assert (perm[N:] == -1).all()
+    t, h, w = perm[:N] // HW, (perm[:N] % HW) // Wd, perm[:N] % Wd
+    assert (t[:HW] == 0).all() and (h[:HW] * Wd + w[:HW] == np.arange(HW)).all()
+    runs = (h[HW:] * Wd + w[HW:]).reshape(HW, T - 1)             # one run of T-1 slots per position
+    assert (runs == np.arange(HW)[:, None]).all()
+    assert (t[HW:].reshape(HW, T - 1) == np.arange(1, T)[None, :]).all()
+
+
+def test_layout1_counts_match_keep_matrix_and_total():
+    # the brute-force tile counts under layout 1, recomputed from the dense keep
+    # matrix permuted by the order, and the total against the kept-pair routine
+    grid, unit = (5, 4, 6), (1, 1, 1)
+    spec = dict(W.mask_spec("temporal", sink=1, rh=1, rw=2), layout=1)
+    n_slots, B = 128, 32
+    perm = oracle.tile_major_order(grid, unit, n_slots, layout=1)
+    km = oracle.keep_matrix(spec, grid, unit).astype(np.int64)
+    real = perm >= 0
+    kp = np.zeros((n_slots, n_slots), dtype=np.int64)
+    kp[np.ix_(real, real)] = km[np.ix_(perm[real], perm[real])]
+    ref = kp.reshape(n_slots // B, B, n_slots // B, B).sum(axis=(1, 3))
+    counts, real_q = oracle.tile_counts(spec, grid, unit, n_slots, B, B)
+    assert (counts == ref).all()
+    assert real_q.sum() == np.prod(grid)
+    assert counts.sum() == oracle.kept_pairs(spec, grid, unit)
+    spec0 = dict(spec, layout=0)
+    c0, _ = oracle.tile_counts(spec0, grid, unit, n_slots, B, B)
+    assert c0.sum() == counts.sum()                                # the order does not change the pairs
+
+
+def test_layout1_temporal_keys_form_bands():
+    # a temporal head's kept keys past frame 0 are one contiguous band per
+    # kept latent row: at most 2 rh + 1 runs per query
+    grid = (6, 7, 9)
+    T, H, Wd = grid
+    HW = H * Wd
+    rh, rw = 1, 2
+    spec = dict(W.mask_spec("temporal", sink=1, rh=rh, rw=rw), layout=1)
+    perm = oracle.tile_major_order(grid, (1, 1, 1), T * HW, layout=1)
+    km = oracle.keep_matrix(spec, grid, (1, 1, 1))
+    for q in (0, 17, 3 * HW + 40, T * HW - 1):
+        row = km[q, perm[HW:]].astype(np.int8)                    # keys of frames >= 1 in layout order
+        starts = int(((row[1:] == 1) & (row[:-1] == 0)).sum() + row[0])
+        hq = (q % HW) // Wd
+        assert starts == min(hq + rh, H - 1) - max(hq - rh, 0) + 1
+        assert km[q, perm[:HW]].all()                               # the sink keeps all of frame 0

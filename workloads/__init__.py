@@ -35,7 +35,7 @@ import numpy as np
 MASK_KINDS = {"full": 0, "spatial": 1, "temporal": 2, "sta": 3, "stripe": 4}
 
 SPEC_KEYS = ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-             "Tw", "To", "Ts", "Sw", "So", "Ss")
+             "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")
 
 
 def mask_spec(kind: str, sink: int = 0, **params) -> Dict[str, int]:
@@ -48,6 +48,9 @@ def mask_spec(kind: str, sink: int = 0, **params) -> Dict[str, int]:
     kt,kh,kw STA window, counted in 3D units (clamped to the unit grid)
     Tw,To,Ts,Sw,So,Ss  stripe width / offset / stride, inter-frame (T*) and
              intra-frame (S*, over s = h*W + w)
+    layout   token order of the head: 0 tile-major over 3D units, 1 frame 0
+             first, then every spatial position with its other frames
+             (temporal heads only)
     """
     if kind not in MASK_KINDS:
         raise ValueError(f"unknown mask kind {kind!r}")
