@@ -45,6 +45,7 @@ LAUNCHES = {"plan_build": 3, "plan_build_stripe": 4, "permute": 1, "unpermute": 
 
 WORKLOADS = {
     "svg_wan720p": W.svg_wan720p,
+    "svg_wan720p_temporal_f0": lambda: W.svg_wan720p(temporal_layout=1),
     "tiny": W.tiny,
     "sta_hunyuan720p": W.sta_hunyuan720p,
     "stripe_wan720p": W.stripe_wan720p,

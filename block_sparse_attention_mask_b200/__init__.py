@@ -41,7 +41,7 @@ class VsaError(RuntimeError):
 class vsa_mask_spec(ctypes.Structure):
     _fields_ = [(k, ctypes.c_int32) for k in
                 ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-                 "Tw", "To", "Ts", "Sw", "So", "Ss")]
+                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")]
 
 
 class vsa_plan_info_t(ctypes.Structure):
@@ -70,6 +70,7 @@ def _load() -> ctypes.CDLL:
         "vsa_plan_tile_map": ([vp, vp, sz, vp], i32),
         "vsa_plan_tile_counts": ([vp, vp, sz, vp], i32),
         "vsa_plan_perm": ([vp, vp, sz, vp], i32),
+        "vsa_plan_layout_perm": ([vp, i32, vp, sz, vp], i32),
         "vsa_plan_exec_steps": ([vp, vp, sz, vp], i32),
         "vsa_plan_kept_pairs": ([vp, vp, sz, vp], i32),
         "vsa_plan_destroy": ([vp], i32),
@@ -183,6 +184,14 @@ def vsa_plan_perm(plan: int, stream=None) -> np.ndarray:
     return out
 
 
+def vsa_plan_layout_perm(plan: int, layout: int, stream=None) -> np.ndarray:
+    info = vsa_plan_info(plan)
+    out = np.empty(info["n_slots"], dtype=np.int32)
+    _check(_lib.vsa_plan_layout_perm(plan, int(layout), out.ctypes.data, out.size, _stream(stream)),
+           "vsa_plan_layout_perm")
+    return out
+
+
 def vsa_plan_exec_steps(plan: int, stream=None) -> np.ndarray:
     info = vsa_plan_info(plan)
     out = np.empty(info["num_heads"], dtype=np.int64)
@@ -282,8 +291,8 @@ class Plan:
     def tile_counts(self, stream=None) -> np.ndarray:
         return vsa_plan_tile_counts(self.handle, stream)
 
-    def perm(self, stream=None) -> np.ndarray:
-        return vsa_plan_perm(self.handle, stream)
+    def perm(self, stream=None, layout: int = 0) -> np.ndarray:
+        return vsa_plan_layout_perm(self.handle, layout, stream)
 
     def exec_steps(self, stream=None) -> np.ndarray:
         return vsa_plan_exec_steps(self.handle, stream)

@@ -437,6 +437,62 @@ __device__ __forceinline__ void box_row_bits(const vsa_mask_spec& m, const vsa_d
     }
 }
 
+// Keep bits of query row q for kv tile kv of a frame-0-first head (temporal or
+// full mask): the frame-0 keys of the tile come in runs along w inside one
+// latent row, kept by the sink or by the w window; every other key sits in a
+// run of frames of one spatial position, all kept or none.
+template <int BK>
+__device__ __forceinline__ void f0_row_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                            int kv, uint32_t (&words)[BK / 32])
+{
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) words[wi] = 0u;
+    if (!q.real) return;
+    const long long HW = (long long)d.H * d.W, N = HW * d.T;
+    const long long p0 = (long long)kv * BK, p1 = p0 + BK;
+    const bool all_keys = m.kind == VSA_MASK_FULL;
+    auto set_range = [&](int lo, int hi) {          // tile bits [lo, hi), 0 <= lo < hi <= BK
+#pragma unroll
+        for (int wi = 0; wi < BK / 32; ++wi) {
+            const int a = max(lo, 32 * wi), b = min(hi, 32 * wi + 32);
+            if (a < b) words[wi] |= (b - a == 32 ? 0xFFFFFFFFu : ((1u << (b - a)) - 1u)) << (a - 32 * wi);
+        }
+    };
+    long long p = p0;
+    while (p < p1 && p < HW) {                      // frame 0
+        const int h = (int)(p / d.W), w = (int)(p - (long long)h * d.W);
+        const int len = (int)min((long long)(d.W - w), min(p1, HW) - p);
+        int lo = 0, hi = len;
+        if (!(m.sink || all_keys)) {
+            if (vsa_iabs(h - q.hq) > m.rh) {
+                hi = 0;
+            } else {
+                lo = max(q.wq - m.rw, w) - w;
+                hi = min(q.wq + m.rw + 1, w + len) - w;
+            }
+        }
+        if (lo < hi) set_range((int)(p - p0) + lo, (int)(p - p0) + hi);
+        p += len;
+    }
+    if (d.T > 1 && p < p1 && p < N) {               // frames 1..T-1, position-major
+        const int F = d.T - 1;
+        const long long r = p - HW;
+        const long long pos = r / F;
+        int f = (int)(r - pos * F);
+        int h = (int)(pos / d.W), w = (int)(pos - (long long)h * d.W);
+        while (p < p1 && p < N) {
+            const int len = (int)min((long long)(F - f), min(p1, N) - p);
+            if (all_keys || (vsa_iabs(h - q.hq) <= m.rh && vsa_iabs(w - q.wq) <= m.rw))
+                set_range((int)(p - p0), (int)(p - p0) + len);
+            p += len;
+            f = 0;
+            if (++w == d.W) {
+                w = 0;
+                ++h;
+            }
+        }
+    }
+}
 template <int BK>
 __device__ __forceinline__ void box_row_bits_any(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
                                                  const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
@@ -711,8 +767,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             for (int i = t; i < P.tab_words_s; i += 64) stab[i] = src[i];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
-        // single-box tiles are evaluated by the softmax threads themselves
-        if (d.box_nh == 0) switch (m.kind) {
+        // single-box tiles and frame-0-first heads are evaluated by the softmax threads
+        if (d.box_nh == 0 && m.layout != VSA_LAYOUT_FRAME0_FIRST) switch (m.kind) {
         case VSA_MASK_FULL:
             mask_worker_loop<VSA_MASK_FULL, BK>(m, d, q0, q1, stab, ttab, P.seg, entries, cnt, t, lane, maskbuf,
                                                 BAR_MF(0), BAR_ME(0), ctl);
@@ -750,7 +806,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         if (X == 0) rowctx[row] = vsa_row_init(d, m, (long long)e * kRows + row);
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
 
-        const bool box = d.box_nh > 0;                    // boundary bits computed here, not by mask workers
+        const bool f0 = m.layout == VSA_LAYOUT_FRAME0_FIRST;
+        const bool box = d.box_nh > 0 && !f0;             // boundary bits computed here, not by mask workers
         float m_run = -INFINITY;  // running max of scale*log2(e)*s over this warpgroup's tiles
         float l_run = 0.0f;
         const float sl = P.scale_log2;
@@ -775,6 +832,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 box_row_bits_any<BK>(m, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
                                      (long long)kv * BK < d.Npad, mw);
             }
+            if (bnd && f0) {
+                const vsa_row_ctx q = rowctx[row];
+                f0_row_bits<BK>(m, d, q, VSA_ENTRY_KV(ent), mw);
+            }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
             float s[BK];
@@ -791,7 +852,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             }
 
             if (bnd) {
-                if (!box) {
+                if (!box && !f0) {
                     // keep bits from the mask workers; the slot is released after reading
                     const int slot = kb % kMaskSlots;
                     if (!mbar_wait_warp(BAR_MF(slot), (uint32_t)(kb / kMaskSlots) & 1, ctl)) { ok = false; break; }

@@ -104,6 +104,41 @@ __device__ __forceinline__ long long vsa_token_slot(const vsa_dims& d, int t, in
     return u * d.U + (ot * d.bh + oh) * d.bw + ow;
 }
 
+// Natural coordinates of slot p of a frame-0-first head (VSA_LAYOUT_FRAME0_FIRST):
+// slots [0, HW) are frame 0 in (h,w) order, then position (h,w) in row-major
+// order with its frames 1..T-1; false for padding slots (p >= T*H*W).
+__device__ __forceinline__ bool vsa_slot_coords_f0(const vsa_dims& d, long long p, int& t, int& h, int& w)
+{
+    const long long HW = (long long)d.H * d.W;
+    if (p < HW) {
+        t = 0;
+        h = (int)(p / d.W);
+        w = (int)(p - (long long)h * d.W);
+        return true;
+    }
+    const long long r = p - HW;
+    if (d.T <= 1 || r >= HW * (d.T - 1)) return false;
+    const long long pos = r / (d.T - 1);
+    t = 1 + (int)(r - pos * (d.T - 1));
+    h = (int)(pos / d.W);
+    w = (int)(pos - (long long)h * d.W);
+    return true;
+}
+
+// Slot of the real token (t,h,w) in a frame-0-first head.
+__device__ __forceinline__ long long vsa_token_slot_f0(const vsa_dims& d, int t, int h, int w)
+{
+    const long long pos = (long long)h * d.W + w;
+    return t == 0 ? pos : (long long)d.H * d.W + pos * (d.T - 1) + (t - 1);
+}
+
+// Either layout.
+__device__ __forceinline__ bool vsa_slot_coords_any(const vsa_dims& d, int layout, long long p, int& t, int& h,
+                                                    int& w)
+{
+    return layout == VSA_LAYOUT_FRAME0_FIRST ? vsa_slot_coords_f0(d, p, t, h, w) : vsa_slot_coords(d, p, t, h, w);
+}
+
 __device__ __forceinline__ int vsa_iabs(int x) { return x < 0 ? -x : x; }
 
 // STA along one axis: first unit of the window of query unit uq.
@@ -163,13 +198,13 @@ __device__ __forceinline__ uint32_t vsa_run_bits(const vsa_mask_spec& m, const v
     }
 }
 
-// Query-row context of tile-major slot `slot` for the predicate above.
+// Query-row context of slot `slot` (in the head's layout) for the predicate above.
 __device__ __forceinline__ vsa_row_ctx vsa_row_init(const vsa_dims& d, const vsa_mask_spec& m,
                                                     long long slot)
 {
     vsa_row_ctx q;
     q.tq = q.hq = q.wq = 0;
-    q.real = vsa_slot_coords(d, slot, q.tq, q.hq, q.wq);
+    q.real = vsa_slot_coords_any(d, m.layout, slot, q.tq, q.hq, q.wq);
     q.sq = q.hq * d.W + q.wq;
     q.kk_t = min(m.kt, d.nTt);
     q.kk_h = min(m.kh, d.nTh);

@@ -1,8 +1,10 @@
-// Token permutation between the natural (t,h,w) order and the tile-major
-// order of 3D units, with zero padding ("Video diffusion long-sequence
-// attention and sparsity", section 7.2: the permutation is one [N, d] gather;
-// "Parameterized Stripe Attention", key design 2: hierarchical layout with
-// 3D padding).  HBM-bound copies: every row of D bf16 values moves as 16-byte
+// Token permutation between the natural (t,h,w) order and each head's layout:
+// the tile-major order of 3D units with zero padding ("Video diffusion
+// long-sequence attention and sparsity", section 7.2: the permutation is one
+// [N, d] gather; "Parameterized Stripe Attention", key design 2: hierarchical
+// layout with 3D padding), or the frame-0-first position-major order of
+// temporal heads ("Sparse VideoGen: accelerating video diffusion attention on
+// TPU", "arranging tokens for efficient temporal access").  HBM-bound copies: every row of D bf16 values moves as 16-byte
 // vectors, a warp covers 2 rows (D = 128) or 4 rows (D = 64) per step, and
 // the grid is a multiple of the SM count with a grid-stride loop.
 #include <cuda_runtime.h>
@@ -12,8 +14,8 @@
 namespace {
 
 template <int D>
-__global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, long long rows,
-                                                      const uint4* __restrict__ in,
+__global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                                      long long rows, const uint4* __restrict__ in,
                                                       uint4* __restrict__ out)
 {
     constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
@@ -27,7 +29,8 @@ __global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, long long rows
         const long long p = r - bh * d.Nslots;
         int t = 0, h = 0, w = 0;
         uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (vsa_slot_coords(d, p, t, h, w)) {
+        const int layout = __ldg(&specs[bh % d.heads].layout);
+        if (vsa_slot_coords_any(d, layout, p, t, h, w)) {
             const long long n = ((long long)t * d.H + h) * d.W + w;
             val = __ldg(in + (bh * d.N + n) * VPR + v);
         }
@@ -36,8 +39,8 @@ __global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, long long rows
 }
 
 template <int D>
-__global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, long long rows,
-                                                        const uint4* __restrict__ in,
+__global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                                        long long rows, const uint4* __restrict__ in,
                                                         uint4* __restrict__ out)
 {
     constexpr int VPR = D * 2 / 16;
@@ -53,7 +56,9 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, long long ro
         const int t = (int)(n / HW);
         const int rem = (int)(n - (long long)t * HW);
         const int h = rem / d.W, w = rem - (rem / d.W) * d.W;
-        const long long p = vsa_token_slot(d, t, h, w);
+        const long long p = __ldg(&specs[bh % d.heads].layout) == VSA_LAYOUT_FRAME0_FIRST
+                                ? vsa_token_slot_f0(d, t, h, w)
+                                : vsa_token_slot(d, t, h, w);
         out[r * VPR + v] = __ldg(in + (bh * d.Nslots + p) * VPR + v);
     }
 }
@@ -90,11 +95,11 @@ int launch(bool forward, vsa_plan_t plan, const void* in, void* out, int B, int 
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     cudaStream_t s = (cudaStream_t)stream;
     if (forward) {
-        if (D == 128) permute_kernel<128><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
-        else permute_kernel<64><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+        if (D == 128) permute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
+        else permute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
     } else {
-        if (D == 128) unpermute_kernel<128><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
-        else unpermute_kernel<64><<<grid, threads, 0, s>>>(d, rows, (const uint4*)in, (uint4*)out);
+        if (D == 128) unpermute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
+        else unpermute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
     }
     return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }

@@ -75,6 +75,51 @@ __device__ bool tile_box(const vsa_dims& d, int tile, int B, int i, Box& bx, boo
     return bx.t0 < bx.t1 && bx.h0 < bx.h1 && bx.w0 < bx.w1;
 }
 
+// Boxes of slots [p0, p0 + B) of a frame-0-first head (VSA_LAYOUT_FRAME0_FIRST):
+// the frame-0 part is a run of (h,w) positions in row-major order (part of a
+// row, whole rows, part of a row); the rest is a run of (position, frame)
+// pairs with frames fastest (part of one position's frames, whole positions
+// with frames 1..T-1, part of one position's frames).  At most 8 boxes; sets
+// pad when the range reaches past the T*H*W real tokens.
+__device__ int f0_tile_boxes(const vsa_dims& d, long long p0, int B, Box* bx, bool& pad)
+{
+    const long long HW = (long long)d.H * d.W, N = HW * d.T, p1 = p0 + B;
+    int n = 0;
+    if (p1 > N) pad = true;
+    // positions [a, b) of the row-major (h,w) order, with frames [t0, t1)
+    auto add_positions = [&](long long a, long long b, int t0, int t1) {
+        while (a < b) {
+            const int h = (int)(a / d.W), w = (int)(a - (long long)h * d.W);
+            if (w == 0 && b - a >= d.W) {
+                const int rows = (int)((b - a) / d.W);
+                bx[n++] = Box{t0, t1, h, h + rows, 0, d.W};
+                a += (long long)rows * d.W;
+            } else {
+                const int len = (int)min((long long)(d.W - w), b - a);
+                bx[n++] = Box{t0, t1, h, h + 1, w, w + len};
+                a += len;
+            }
+        }
+    };
+    if (p0 < HW) add_positions(p0, min(p1, HW), 0, 1);
+    if (d.T > 1 && p1 > HW && p0 < N) {
+        const long long F = d.T - 1;
+        long long r0 = max(p0, HW) - HW;
+        const long long r1 = min(p1, N) - HW;
+        if (r0 % F) {                              // the tail of one position's frames
+            const long long pos = r0 / F;
+            const long long end = min(r1, (pos + 1) * F);
+            add_positions(pos, pos + 1, 1 + (int)(r0 - pos * F), 1 + (int)(end - pos * F));
+            r0 = end;
+        }
+        const long long pa = r0 / F, pb = r1 / F;
+        if (pb > pa) add_positions(pa, pb, 1, d.T);  // whole positions
+        if (r1 > pb * F && pb * F >= r0)           // the head of one position's frames
+            add_positions(pb, pb + 1, 1, 1 + (int)(r1 - pb * F));
+    }
+    return n;
+}
+
 __device__ __forceinline__ bool rel_t(const vsa_mask_spec& m, const vsa_dims& d, int tq, int tk)
 {
     switch (m.kind) {
@@ -173,12 +218,16 @@ __device__ void classify_boxes(const vsa_mask_spec& m, const vsa_dims& d, const 
         return;
     }
     bool anyt = false, allt = true;
-    for (int tq = A.t0; tq < A.t1; ++tq)
-        for (int tk = tk0; tk < B.t1; ++tk) {
-            const bool r = rel_t(m, d, tq, tk);
-            anyt = anyt || r;
-            allt = allt && r;
-        }
+    if (m.kind == VSA_MASK_SVG_TEMPORAL || m.kind == VSA_MASK_FULL) {
+        anyt = true;                     // no relation on t
+    } else {
+        for (int tq = A.t0; tq < A.t1; ++tq)
+            for (int tk = tk0; tk < B.t1; ++tk) {
+                const bool r = rel_t(m, d, tq, tk);
+                anyt = anyt || r;
+                allt = allt && r;
+            }
+    }
     bool anys = false, alls = false;
     if (anyt || allt) rel_s(m, d, sbits, A, B, anys, alls);
     any = sinkk || (anyt && anys);
@@ -196,6 +245,23 @@ __global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ sp
     const int a = (int)(rem / d.nK), b = (int)(rem - (long long)a * d.nK);
     const vsa_mask_spec m = specs[head];
     const uint32_t* sb = sbits ? sbits + (size_t)head * d.sbits_words : nullptr;
+    if (m.layout == VSA_LAYOUT_FRAME0_FIRST) {
+        Box qb[8], kb[8];
+        bool qpad = false, kpad = false;
+        const int nq = f0_tile_boxes(d, (long long)a * d.Bq, d.Bq, qb, qpad);
+        const int nk = f0_tile_boxes(d, (long long)b * d.Bk, d.Bk, kb, kpad);
+        bool any = false, all = true;
+        for (int i = 0; i < nq && !(any && !all); ++i)
+            for (int j = 0; j < nk; ++j) {
+                bool ba, bl;
+                classify_boxes(m, d, sb, qb[i], kb[j], ba, bl);
+                any = any || ba;
+                all = all && bl;
+                if (any && !all) break;
+            }
+        map[idx] = (nq > 0 && any) ? ((all && !kpad && nk > 0) ? VSA_TILE_FULL : VSA_TILE_BOUNDARY) : VSA_TILE_EMPTY;
+        return;
+    }
     const int nqb = d.Bq <= d.U ? 1 : d.Bq / d.U;
     const int nkb = d.Bk <= d.U ? 1 : d.Bk / d.U;
 
@@ -324,7 +390,8 @@ __global__ void __launch_bounds__(256) kept_pairs_kernel(vsa_dims d, const vsa_m
 {
     extern __shared__ uint32_t tabs[];
     const int head = blockIdx.y;
-    const vsa_mask_spec m = specs[head];
+    vsa_mask_spec m = specs[head];
+    m.layout = VSA_LAYOUT_TILE_MAJOR;   // the total does not depend on the order; the runs are tile-major
     const int ws = (m.kind == VSA_MASK_STRIPE) ? d.sbits_words : 0;
     const int wt = (m.kind == VSA_MASK_STRIPE) ? vsa_ttab_words(d.T) : 0;
     uint32_t* stab = tabs;
@@ -348,12 +415,12 @@ __global__ void __launch_bounds__(256) kept_pairs_kernel(vsa_dims d, const vsa_m
     if ((threadIdx.x & 31) == 0 && cnt) atomicAdd(&kept[head], cnt);
 }
 
-__global__ void perm_kernel(vsa_dims d, int32_t* __restrict__ perm)
+__global__ void perm_kernel(vsa_dims d, int layout, int32_t* __restrict__ perm)
 {
     const long long p = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (p >= d.Nslots) return;
     int t, h, w;
-    perm[p] = vsa_slot_coords(d, p, t, h, w) ? (int32_t)(((long long)t * d.H + h) * d.W + w) : -1;
+    perm[p] = vsa_slot_coords_any(d, layout, p, t, h, w) ? (int32_t)(((long long)t * d.H + h) * d.W + w) : -1;
 }
 
 bool tile_fits_unit(int B, int U, int bh, int bw)
@@ -395,6 +462,9 @@ static int validate_spec(const vsa_mask_spec& m)
 {
     if (m.kind < VSA_MASK_FULL || m.kind > VSA_MASK_STRIPE) return VSA_ERR_INVALID_ARG;
     if (m.sink != 0 && m.sink != 1) return VSA_ERR_INVALID_ARG;
+    if (m.layout != VSA_LAYOUT_TILE_MAJOR && m.layout != VSA_LAYOUT_FRAME0_FIRST) return VSA_ERR_INVALID_ARG;
+    if (m.layout == VSA_LAYOUT_FRAME0_FIRST && m.kind != VSA_MASK_SVG_TEMPORAL && m.kind != VSA_MASK_FULL)
+        return VSA_ERR_UNSUPPORTED;
     const int lim = 1 << 20;
     switch (m.kind) {
     case VSA_MASK_SVG_SPATIAL:
@@ -658,14 +728,20 @@ extern "C" int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n,
 
 extern "C" int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream)
 {
+    return vsa_plan_layout_perm(plan, VSA_LAYOUT_TILE_MAJOR, host_dst, n, stream);
+}
+
+extern "C" int vsa_plan_layout_perm(vsa_plan_t plan, int layout, int32_t* host_dst, size_t n, void* stream)
+{
     if (!plan || !host_dst || n < (size_t)plan->d.Nslots) return VSA_ERR_INVALID_ARG;
+    if (layout != VSA_LAYOUT_TILE_MAJOR && layout != VSA_LAYOUT_FRAME0_FIRST) return VSA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     int32_t* tmp = nullptr;
     if (cudaMalloc(&tmp, sizeof(int32_t) * plan->d.Nslots) != cudaSuccess) {
         cudaGetLastError();
         return VSA_ERR_OOM;
     }
-    perm_kernel<<<blocks_for(plan->d.Nslots, 256), 256, 0, s>>>(plan->d, tmp);
+    perm_kernel<<<blocks_for(plan->d.Nslots, 256), 256, 0, s>>>(plan->d, layout, tmp);
     cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess)
         e = cudaMemcpyAsync(host_dst, tmp, sizeof(int32_t) * plan->d.Nslots, cudaMemcpyDeviceToHost, s);

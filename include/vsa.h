@@ -93,7 +93,23 @@ typedef struct {
     int32_t kt, kh, kw;      /* STA window in units (>= 1)                       */
     int32_t Tw, To, Ts;      /* stripe, inter-frame: width >= 1, offset, stride >= 1 */
     int32_t Sw, So, Ss;      /* stripe, intra-frame: width >= 1, offset, stride >= 1 */
+    int32_t layout;          /* vsa_layout: token order of this head (see below)   */
 } vsa_mask_spec;
+
+/* Token order of a head inside the [B, heads, n_slots, D] tensors.
+   VSA_LAYOUT_TILE_MAJOR: tile-major over the 3D units (bt,bh,bw), padded per
+     axis ("Parameterized Stripe Attention", key design 2).
+   VSA_LAYOUT_FRAME0_FIRST: frame 0 in (h,w) row-major order, then every
+     spatial position (h,w) in row-major order with its frames 1..T-1 in
+     order; no padding inside, slots past T*H*W are padding.  This is the
+     temporal-head permutation of "Sparse VideoGen: accelerating video
+     diffusion attention on TPU" ("arranging tokens for efficient temporal
+     access"), with the frame-0 sink kept in front so that it does not put a
+     kept key in every tile.  Allowed for temporal and full heads only
+     (VSA_ERR_UNSUPPORTED otherwise).  vsa_permute / vsa_unpermute and the
+     tile map follow each head's layout; the attention output is the same
+     set of rows in another order. */
+typedef enum { VSA_LAYOUT_TILE_MAJOR = 0, VSA_LAYOUT_FRAME0_FIRST = 1 } vsa_layout;
 
 typedef struct vsa_plan_s* vsa_plan_t;
 
@@ -149,6 +165,12 @@ int vsa_plan_tile_counts(vsa_plan_t plan, int64_t* host_counts, size_t n, void* 
 
 /* Synchronous: perm[slot] = natural token index or -1 (padding), n >= n_slots. */
 int vsa_plan_perm(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream);
+
+/* The same for either layout (vsa_layout): perm[slot] = natural token index
+   (t*H + h)*W + w or -1 for padding, n >= n_slots.  VSA_ERR_INVALID_ARG for an
+   unknown layout.  Synchronous on `stream`; allocates and frees a device
+   buffer of n_slots int32. */
+int vsa_plan_layout_perm(vsa_plan_t plan, int layout, int32_t* host_dst, size_t n, void* stream);
 
 /* Synchronous: number of executed (kv tile, 128-row query block) steps per
  * head, host_dst[h]; the attention kernel runs one tensor-core tile per step. */

@@ -51,7 +51,10 @@ class GpuRun:
         self.o_dev = o                                  # natural order, on the GPU
         self.lse_tm = lse.cpu().numpy().astype(np.float64)
         self.perm = oracle.tile_major_order(self.grid, w.unit, self.plan.n_slots)
-        self.inv = inverse_perm(self.perm, w.N)
+        # each head's own token order (its layout field)
+        self.perms = [oracle.tile_major_order(self.grid, w.unit, self.plan.n_slots,
+                                              layout=int(spec.get("layout", 0))) for spec in w.specs]
+        self.invs = [inverse_perm(p, w.N) for p in self.perms]
 
     def o_rows(self, b: int, h: int, rows) -> np.ndarray:
         import torch
@@ -59,7 +62,7 @@ class GpuRun:
         return self.o_dev[b, h].index_select(0, idx).float().cpu().numpy().astype(np.float64)
 
     def lse_natural(self, b: int, h: int) -> np.ndarray:
-        return self.lse_tm[b, h][self.inv]
+        return self.lse_tm[b, h][self.invs[h]]
 
     def compare_rows(self, h: int, rows, b: int = 0):
         """Oracle vs GPU on natural query rows of head h; returns (max, mean, lse max)."""

@@ -65,6 +65,8 @@ def test_plan_create_rejects_bad_arguments_on_host():
         ([dict(W.mask_spec("stripe", Tw=1, Ts=1, Sw=1, Ss=1), Ts=0)], dict(), -1),
         ([W.mask_spec("temporal", rh=-1, rw=0)], dict(), -1),
         ([W.mask_spec("stripe", Tw=1, Ts=2, Sw=1, Ss=3)], dict(grid=(2, 300, 300), unit=(1, 8, 8)), -2),
+        ([dict(ok, layout=1)], dict(), -2),                # frame-0-first order: temporal / full heads only
+        ([dict(ok, layout=2)], dict(), -1),                # unknown layout
     ]
     for specs, kw, want in cases:
         rc, handle = _create_raw(specs, **kw)
@@ -79,6 +81,7 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_plan_tile_map(None, None, 0, None) == -1
     assert L.vsa_plan_tile_counts(None, None, 0, None) == -1
     assert L.vsa_plan_perm(None, None, 0, None) == -1
+    assert L.vsa_plan_layout_perm(None, 0, None, 0, None) == -1
     assert L.vsa_plan_exec_steps(None, None, 0, None) == -1
     assert L.vsa_plan_destroy(None) == -1
     assert L.vsa_permute(None, None, None, 1, 128, None) == -1

@@ -78,6 +78,28 @@ def test_svg_wan720p():
     assert kept.tolist() == [80 * 3600 ** 2] * 5 + [21 * 3600 ** 2 + 420 * 465 * 1288] * 5
 
 
+def test_svg_wan720p_temporal_frame0_first():
+    # the temporal heads in the frame-0-first, position-major order: maps of
+    # sampled q tiles against the oracle in that order, outputs of sampled
+    # rows, and the layout-invariant kept pairs; far fewer executed tiles
+    w = W.svg_wan720p(temporal_layout=1)
+    counts, _ = _check(w, [0, 5, 9], 96, [5, 9], qtiles_per_head=8)
+    for h in range(5):
+        assert counts[h].tolist() == [324900, 12000, 60000]
+    base = W.svg_wan720p()
+    import block_sparse_attention_mask_b200 as vsa
+    plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile)
+    plan0 = vsa.Plan(list(base.specs), (base.T, base.H, base.W), base.unit, base.q_tile, base.kv_tile)
+    try:
+        assert (plan.kept_pairs() == plan0.kept_pairs()).all()
+        steps, steps0 = plan.exec_steps(), plan0.exec_steps()
+        assert (steps[:5] == steps0[:5]).all()
+        assert int(steps[5:].sum()) < int(steps0[5:].sum())
+    finally:
+        plan.close()
+        plan0.close()
+
+
 def test_sta_hunyuan720p():
     w = W.sta_hunyuan720p()
     counts, _ = _check(w, [0, 11, 23], 96, [0])

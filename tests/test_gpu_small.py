@@ -44,6 +44,17 @@ CASES = {
                       [S("stripe", 0, Tw=1, To=9, Ts=1000, Sw=1, So=0, Ss=1000), S("spatial", 0, rt=0)]),
     "sta_sink_d64": ((6, 16, 16), (2, 8, 8), 128, 128, 64,
                      [S("sta", 1, kt=1, kh=1, kw=1), S("sta", 0, kt=3, kh=3, kw=3)]),
+    # frame-0-first heads next to tile-major ones in one plan
+    "frame0_first_mixed": ((5, 13, 20), (1, 8, 16), 128, 128, 128,
+                           [S("temporal", 1, rh=2, rw=3, layout=1), S("temporal", 0, rh=1, rw=5, layout=1),
+                            S("full", 0, layout=1), S("spatial", 1, rt=1)]),
+    "frame0_first_q64_k64_d64": ((4, 9, 11), (1, 8, 8), 64, 64, 64,
+                                 [S("temporal", 1, rh=1, rw=2, layout=1), S("temporal", 1, rh=0, rw=0, layout=1),
+                                  S("temporal", 0, rh=2, rw=1)]),
+    "frame0_first_ragged": ((3, 7, 9), (1, 1, 1), 128, 64, 64,
+                            [S("temporal", 1, rh=1, rw=1, layout=1), S("full", 1, layout=1)]),
+    "frame0_first_one_frame": ((1, 8, 16), (1, 8, 16), 128, 128, 128,
+                               [S("temporal", 0, rh=1, rw=2, layout=1), S("temporal", 1, rh=1, rw=2, layout=1)]),
 }
 
 
@@ -90,6 +101,9 @@ def test_exec_steps_follow_the_map(run):
 
 def test_perm_matches_oracle(run):
     assert (run.plan.perm() == run.perm).all()
+    for layout in (0, 1):
+        want = oracle.tile_major_order(run.grid, run.w.unit, run.plan.n_slots, layout=layout)
+        assert (run.plan.perm(layout=layout) == want).all()
 
 
 def test_permute_bit_exact_and_round_trip(run):
@@ -101,8 +115,9 @@ def test_permute_bit_exact_and_round_trip(run):
     xt = vsa.permute(run.plan, xd)
     got = xt.view(torch.int16).cpu().numpy().view(np.uint16)
     want = np.zeros((w.B, w.heads, run.plan.n_slots, w.D), dtype=np.uint16)
-    real = run.perm >= 0
-    want[:, :, real] = x[:, :, run.perm[real]]
+    for h in range(w.heads):
+        real = run.perms[h] >= 0
+        want[:, h, real] = x[:, h, run.perms[h][real]]
     assert (got == want).all()
     back = vsa.unpermute(run.plan, xt)
     assert torch.equal(back.view(torch.int16), xd.view(torch.int16))
