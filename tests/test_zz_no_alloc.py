@@ -49,6 +49,8 @@ CALLS = [
       S("spatial", 1, rt=1), S("sta", 0, kt=3, kh=1, kw=1)], (5, 13, 20), (1, 8, 16), 128, 128),
     # no stripe head, other tile shape
     (list(W.svg_wan720p().specs), (21, 45, 80), (1, 8, 8), 64, 64),
+    # temporal heads in the frame-0-first order
+    (list(W.svg_wan720p(temporal_layout=1).specs), (21, 45, 80), (1, 8, 16), 128, 128),
 ]
 
 
