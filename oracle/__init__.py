@@ -29,7 +29,7 @@ _lib = None
 class _Mask(ctypes.Structure):
     _fields_ = [(k, ctypes.c_int32) for k in
                 ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")]
+                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout", "tile_round")]
 
 
 class _Grid(ctypes.Structure):
@@ -192,3 +192,54 @@ def tile_map(spec, grid, unit, n_slots: int, Bq: int, Bk: int,
 def kept_pairs(spec, grid, unit=(1, 1, 1), nthreads: Optional[int] = None) -> int:
     return int(_load().orc_kept_pairs(ctypes.byref(_mask(spec)), ctypes.byref(_grid(grid, unit)),
                                       int(nthreads or default_threads())))
+
+
+def rounded_tile_map(spec, grid, unit, n_slots: int, Bq: int, Bk: int,
+                     qtiles: Optional[Iterable[int]] = None, nthreads: Optional[int] = None
+                     ) -> np.ndarray:
+    """Tile-aligned rounding of the mask ("Sparse VideoGen: accelerating video
+    diffusion attention on TPU", "aligning the sparse mask with execution",
+    B3).  Reading: a tile pair with some kept (real query, real key) pairs
+    becomes kept whole when at least half of its real pairs are kept and is
+    dropped otherwise, which rounds outward and inward in balance; a kept kv
+    tile holding padding slots stays class 1, its padding masked.  Classes
+    from the brute-force counts in the head's token order."""
+    counts, real_q = tile_counts(spec, grid, unit, n_slots, Bq, Bk, qtiles, nthreads)
+    perm = tile_major_order(grid, unit, n_slots, layout=int(spec.get("layout", 0)))
+    real_k = (perm.reshape(-1, Bk) >= 0).sum(axis=1)
+    pairs = real_q[:, None] * real_k[None, :]
+    kept = (counts > 0) & (2 * counts >= pairs)
+    return np.where(kept, np.where(real_k[None, :] == Bk, 2, 1), 0).astype(np.int8)
+
+
+def attention_rows_rounded(spec, grid, unit, n_slots: int, Bq: int, Bk: int, D: int, scale: float,
+                           q: np.ndarray, k: np.ndarray, v: np.ndarray, rows) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 softmax(scale q k^T) v of natural query rows under the rounded mask:
+    query n keeps every real key of every kv tile that the rounded map keeps for
+    n's q tile.  q, k, v are one head's bf16 bits [N, D] in natural order."""
+    perm = tile_major_order(grid, unit, n_slots, layout=int(spec.get("layout", 0)))
+    n_tok = int(np.prod(grid))
+    slot_of = np.full(n_tok, -1, dtype=np.int64)
+    real = perm >= 0
+    slot_of[perm[real]] = np.nonzero(real)[0]
+    rows = np.asarray(rows, dtype=np.int64)
+    qt_of = slot_of[rows] // Bq
+    qts = np.unique(qt_of)
+    cls = rounded_tile_map(spec, grid, unit, n_slots, Bq, Bk, qts)
+    f64 = lambda b: (np.asarray(b, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+    qf, kf, vf = f64(q), f64(k), f64(v)
+    o = np.zeros((len(rows), D))
+    lse = np.full(len(rows), -np.inf)
+    for i, (n, qt) in enumerate(zip(rows, qt_of)):
+        kv_tiles = np.nonzero(cls[np.searchsorted(qts, qt)] != 0)[0]
+        if len(kv_tiles) == 0:
+            continue
+        slots = (kv_tiles[:, None] * Bk + np.arange(Bk)[None, :]).ravel()
+        keys = perm[slots]
+        keys = keys[keys >= 0]
+        s = (kf[keys] @ qf[n]) * scale
+        mx = s.max()
+        p = np.exp(s - mx)
+        o[i] = (p @ vf[keys]) / p.sum()
+        lse[i] = mx + np.log(p.sum())
+    return o, lse

@@ -57,6 +57,7 @@
 typedef struct {
     int32_t kind, sink, rt, rh, rw, kt, kh, kw, Tw, To, Ts, Sw, So, Ss;
     int32_t layout;   /* token order of the head: 0 tile-major, 1 frame 0 first */
+    int32_t tile_round;  /* unused here: the rounded mask is built in Python from the counts */
 } orc_mask;
 
 typedef struct {

@@ -401,3 +401,81 @@ def test_layout1_temporal_keys_form_bands():
         hq = (q % HW) // Wd
         assert starts == min(hq + rh, H - 1) - max(hq - rh, 0) + 1
         assert km[q, perm[:HW]].all()                               # the sink keeps all of frame 0
+
+
+# --- tile-aligned rounding (lossy mode) ---------------------------------------------
+
+
+def _rounded_from_keep_matrix(spec, grid, unit, n_slots, B):
+    # the rounding rule restated on the dense keep matrix permuted into the head's order
+    perm = oracle.tile_major_order(grid, unit, n_slots, layout=int(spec.get("layout", 0)))
+    km = oracle.keep_matrix(spec, grid, unit).astype(np.int64)
+    real = perm >= 0
+    kp = np.zeros((n_slots, n_slots), dtype=np.int64)
+    kp[np.ix_(real, real)] = km[np.ix_(perm[real], perm[real])]
+    cnt = kp.reshape(n_slots // B, B, n_slots // B, B).sum(axis=(1, 3))
+    rq = real.reshape(-1, B).sum(axis=1)
+    pairs = rq[:, None] * rq[None, :]
+    keep = (cnt > 0) & (2 * cnt >= pairs)
+    return np.where(keep, np.where(rq[None, :] == B, 2, 1), 0), cnt, pairs
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_rounded_map_rule_and_exact_tiles(layout):
+    grid, unit, n_slots, B = (5, 4, 6), (1, 2, 3), 128, 32
+    spec = dict(W.mask_spec("temporal", sink=1, rh=1, rw=1), layout=layout, tile_round=1)
+    got = oracle.rounded_tile_map(spec, grid, unit, n_slots, B, B)
+    want, cnt, pairs = _rounded_from_keep_matrix(spec, grid, unit, n_slots, B)
+    assert (got == want).all()
+    exact = oracle.tile_map(spec, grid, unit, n_slots, B, B)
+    assert (got[exact == 0] == 0).all() and (got[exact == 2] == 2).all()   # only boundary tiles move
+    assert ((got == 1) <= (exact == 1)).all()
+    moved = exact == 1
+    assert ((got[moved] != 0) == (2 * cnt[moved] >= pairs[moved])).all()
+
+
+def test_rounding_a_full_mask_changes_nothing():
+    grid, unit = (3, 7, 9), (1, 1, 1)
+    spec = dict(W.mask_spec("full"), tile_round=1)
+    assert (oracle.rounded_tile_map(spec, grid, unit, 256, 64, 64) ==
+            oracle.tile_map(spec, grid, unit, 256, 64, 64)).all()
+
+
+def test_rounded_attention_is_exact_for_a_tile_aligned_mask():
+    # spatial |dt| <= 0 with one frame per tile: every tile pair is full or
+    # empty, so rounding must not change a single output
+    grid, unit, B, D = (4, 4, 8), (1, 4, 8), 32, 64
+    spec = W.mask_spec("spatial", sink=0, rt=0)
+    rspec = dict(spec, tile_round=1)
+    w = W.Workload("t", 1, *grid, 1, D, unit, B, B, (spec,))
+    q, k, v = (W.head_tensor(w, x, 0, 0) for x in "qkv")
+    rows = np.arange(int(np.prod(grid)))
+    o1, l1 = oracle.attention_rows(spec, grid, unit, D, w.scale, q, k, v, rows)
+    o2, l2 = oracle.attention_rows_rounded(rspec, grid, unit, 128, B, B, D, w.scale, q, k, v, rows)
+    assert np.allclose(o1, o2, atol=1e-12) and np.allclose(l1, l2, atol=1e-12)
+
+
+def test_rounded_attention_against_dense_reference():
+    # the rounded keep matrix, dense fp64 softmax by hand
+    grid, unit, B, D = (5, 4, 6), (1, 2, 3), 32, 64
+    spec = dict(W.mask_spec("temporal", sink=1, rh=1, rw=1), tile_round=1)
+    cls, _, _ = _rounded_from_keep_matrix(spec, grid, unit, 128, B)
+    perm = oracle.tile_major_order(grid, unit, 128)
+    w = W.Workload("t", 1, *grid, 1, D, unit, B, B, (spec,))
+    q, k, v = (W.head_tensor(w, x, 0, 0) for x in "qkv")
+    f = lambda b: (b.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    qf, kf, vf = f(q), f(k), f(v)
+    N = int(np.prod(grid))
+    slot_of = np.empty(N, dtype=np.int64)
+    slot_of[perm[perm >= 0]] = np.nonzero(perm >= 0)[0]
+    keep = np.zeros((N, N), dtype=bool)
+    for n in range(N):
+        for m in range(N):
+            keep[n, m] = cls[slot_of[n] // B, slot_of[m] // B] != 0
+    s = qf @ kf.T * w.scale
+    s[~keep] = -np.inf
+    mx = s.max(axis=1, keepdims=True)
+    p = np.exp(s - mx)
+    o_ref = (p @ vf) / p.sum(axis=1, keepdims=True)
+    o, _ = oracle.attention_rows_rounded(spec, grid, unit, 128, B, B, D, w.scale, q, k, v, np.arange(N))
+    assert np.abs(o - o_ref).max() < 1e-12

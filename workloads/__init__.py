@@ -35,7 +35,7 @@ import numpy as np
 MASK_KINDS = {"full": 0, "spatial": 1, "temporal": 2, "sta": 3, "stripe": 4}
 
 SPEC_KEYS = ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-             "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")
+             "Tw", "To", "Ts", "Sw", "So", "Ss", "layout", "tile_round")
 
 
 def mask_spec(kind: str, sink: int = 0, **params) -> Dict[str, int]:
@@ -51,6 +51,7 @@ def mask_spec(kind: str, sink: int = 0, **params) -> Dict[str, int]:
     layout   token order of the head: 0 tile-major over 3D units, 1 frame 0
              first, then every spatial position with its other frames
              (temporal heads only)
+    tile_round  1: tile-aligned rounding of the mask (lossy; SVG and full heads)
     """
     if kind not in MASK_KINDS:
         raise ValueError(f"unknown mask kind {kind!r}")
