@@ -46,6 +46,8 @@ LAUNCHES = {"plan_build": 3, "plan_build_stripe": 4, "permute": 1, "unpermute": 
 WORKLOADS = {
     "svg_wan720p": W.svg_wan720p,
     "svg_wan720p_temporal_f0": lambda: W.svg_wan720p(temporal_layout=1),
+    "svg_wan720p_rounded": lambda: W.svg_wan720p(tile_round=1),
+    "svg_wan720p_temporal_f0_rounded": lambda: W.svg_wan720p(temporal_layout=1, tile_round=1),
     "tiny": W.tiny,
     "sta_hunyuan720p": W.sta_hunyuan720p,
     "stripe_wan720p": W.stripe_wan720p,

@@ -41,7 +41,7 @@ class VsaError(RuntimeError):
 class vsa_mask_spec(ctypes.Structure):
     _fields_ = [(k, ctypes.c_int32) for k in
                 ("kind", "sink", "rt", "rh", "rw", "kt", "kh", "kw",
-                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout")]
+                 "Tw", "To", "Ts", "Sw", "So", "Ss", "layout", "tile_round")]
 
 
 class vsa_plan_info_t(ctypes.Structure):

@@ -759,7 +759,13 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // ---------------- mask workers (warps 10, 11) ----------------
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
         const int t = threadIdx.x - kMaskWarp0 * 32;      // rows t and t + 64
-        const vsa_mask_spec m = P.specs[head];
+        const vsa_mask_spec m0 = P.specs[head];
+        // a rounded head keeps whole tiles: only its padding is masked
+        vsa_mask_spec m = m0;
+        if (m0.tile_round) {
+            m.kind = VSA_MASK_FULL;
+            m.sink = 0;
+        }
         const vsa_row_ctx q0 = vsa_row_init(d, m, (long long)e * kRows + t);
         const vsa_row_ctx q1 = vsa_row_init(d, m, (long long)e * kRows + t + 64);
         if (m.kind == VSA_MASK_STRIPE) {
@@ -807,6 +813,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         asm volatile("bar.sync 1, %0;" ::"n"(32 * (kSoftmaxWarps + 2)) : "memory");
 
         const bool f0 = m.layout == VSA_LAYOUT_FRAME0_FIRST;
+        // a rounded head keeps whole tiles: its boundary tiles only mask padding
+        vsa_mask_spec mb = m;
+        if (m.tile_round) {
+            mb.kind = VSA_MASK_FULL;
+            mb.sink = 0;
+        }
         const bool box = d.box_nh > 0 && !f0;             // boundary bits computed here, not by mask workers
         float m_run = -INFINITY;  // running max of scale*log2(e)*s over this warpgroup's tiles
         float l_run = 0.0f;
@@ -829,12 +841,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             if (bnd && box) {
                 const int kv = VSA_ENTRY_KV(ent);
                 const vsa_row_ctx q = rowctx[row];
-                box_row_bits_any<BK>(m, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                box_row_bits_any<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
                                      (long long)kv * BK < d.Npad, mw);
             }
             if (bnd && f0) {
                 const vsa_row_ctx q = rowctx[row];
-                f0_row_bits<BK>(m, d, q, VSA_ENTRY_KV(ent), mw);
+                f0_row_bits<BK>(mb, d, q, VSA_ENTRY_KV(ent), mw);
             }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();

@@ -206,6 +206,54 @@ __device__ void rel_s(const vsa_mask_spec& m, const vsa_dims& d, const uint32_t*
     }
 }
 
+// #{(a, b) : a in [a0,a1), b in [b0,b1), |a - b| <= r}
+__device__ long long pairs_within(int a0, int a1, int b0, int b1, int r)
+{
+    long long n = 0;
+    for (int a = a0; a < a1; ++a) n += max(0, min(b1 - 1, a + r) - max(b0, a - r) + 1);
+    return n;
+}
+
+// Kept pairs over real (A x B), for the masks tile rounding accepts (full,
+// SVG spatial and temporal, with the frame-0 sink): the frame-0 keys of a
+// sink head are all kept, the rest is a product of per-axis pair counts.
+__device__ long long count_kept(const vsa_mask_spec& m, const Box& A, const Box& B)
+{
+    const long long ahw = (long long)(A.h1 - A.h0) * (A.w1 - A.w0);
+    const long long bhw = (long long)(B.h1 - B.h0) * (B.w1 - B.w0);
+    const int at = A.t1 - A.t0;
+    long long kept = 0;
+    int tk0 = B.t0;
+    if (m.sink && B.t0 == 0) {
+        kept += (long long)at * ahw * bhw;
+        tk0 = 1;
+    }
+    if (tk0 >= B.t1) return kept;
+    const int bt = B.t1 - tk0;
+    switch (m.kind) {
+    case VSA_MASK_SVG_SPATIAL:
+        return kept + pairs_within(A.t0, A.t1, tk0, B.t1, m.rt) * ahw * bhw;
+    case VSA_MASK_SVG_TEMPORAL:
+        return kept + (long long)at * bt * pairs_within(A.h0, A.h1, B.h0, B.h1, m.rh) *
+                          pairs_within(A.w0, A.w1, B.w0, B.w1, m.rw);
+    default:
+        return kept + (long long)at * bt * ahw * bhw;
+    }
+}
+
+__device__ __forceinline__ long long box_size(const Box& b)
+{
+    return (long long)(b.t1 - b.t0) * (b.h1 - b.h0) * (b.w1 - b.w0);
+}
+
+// Class of a tile pair under tile-aligned rounding: kept whole when at least
+// half of its real pairs are kept (class 1 if the kv tile holds padding).
+__device__ int8_t rounded_class(long long kept, long long pairs, bool kpad)
+{
+    if (kept == 0 || 2 * kept < pairs) return VSA_TILE_EMPTY;
+    return kpad ? VSA_TILE_BOUNDARY : VSA_TILE_FULL;
+}
+
 // any / all kept over real (A x B).
 __device__ void classify_boxes(const vsa_mask_spec& m, const vsa_dims& d, const uint32_t* sbits,
                                const Box& A, const Box& B, bool& any, bool& all)
@@ -250,6 +298,15 @@ __global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ sp
         bool qpad = false, kpad = false;
         const int nq = f0_tile_boxes(d, (long long)a * d.Bq, d.Bq, qb, qpad);
         const int nk = f0_tile_boxes(d, (long long)b * d.Bk, d.Bk, kb, kpad);
+        if (m.tile_round) {
+            long long kept = 0, nqr = 0, nkr = 0;
+            for (int i = 0; i < nq; ++i) nqr += box_size(qb[i]);
+            for (int j = 0; j < nk; ++j) nkr += box_size(kb[j]);
+            for (int i = 0; i < nq; ++i)
+                for (int j = 0; j < nk; ++j) kept += count_kept(m, qb[i], kb[j]);
+            map[idx] = rounded_class(kept, nqr * nkr, kpad);
+            return;
+        }
         bool any = false, all = true;
         for (int i = 0; i < nq && !(any && !all); ++i)
             for (int j = 0; j < nk; ++j) {
@@ -264,6 +321,27 @@ __global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ sp
     }
     const int nqb = d.Bq <= d.U ? 1 : d.Bq / d.U;
     const int nkb = d.Bk <= d.U ? 1 : d.Bk / d.U;
+    if (m.tile_round) {
+        bool qpad = false, kpad = false;
+        long long kept = 0, nqr = 0, nkr = 0;
+        for (int j = 0; j < nkb; ++j) {
+            Box B;
+            if (tile_box(d, b, d.Bk, j, B, kpad)) nkr += box_size(B);
+            else kpad = true;
+        }
+        for (int i = 0; i < nqb; ++i) {
+            Box A;
+            if (!tile_box(d, a, d.Bq, i, A, qpad)) continue;
+            nqr += box_size(A);
+            for (int j = 0; j < nkb; ++j) {
+                Box B;
+                bool kp = false;
+                if (tile_box(d, b, d.Bk, j, B, kp)) kept += count_kept(m, A, B);
+            }
+        }
+        map[idx] = rounded_class(kept, nqr * nkr, kpad);
+        return;
+    }
 
     bool qpad = false, kpad = false, anyq = false;
     bool any = false, all = true;
@@ -464,6 +542,9 @@ static int validate_spec(const vsa_mask_spec& m)
     if (m.sink != 0 && m.sink != 1) return VSA_ERR_INVALID_ARG;
     if (m.layout != VSA_LAYOUT_TILE_MAJOR && m.layout != VSA_LAYOUT_FRAME0_FIRST) return VSA_ERR_INVALID_ARG;
     if (m.layout == VSA_LAYOUT_FRAME0_FIRST && m.kind != VSA_MASK_SVG_TEMPORAL && m.kind != VSA_MASK_FULL)
+        return VSA_ERR_UNSUPPORTED;
+    if (m.tile_round != 0 && m.tile_round != 1) return VSA_ERR_INVALID_ARG;
+    if (m.tile_round && m.kind != VSA_MASK_FULL && m.kind != VSA_MASK_SVG_SPATIAL && m.kind != VSA_MASK_SVG_TEMPORAL)
         return VSA_ERR_UNSUPPORTED;
     const int lim = 1 << 20;
     switch (m.kind) {

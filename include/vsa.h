@@ -94,7 +94,18 @@ typedef struct {
     int32_t Tw, To, Ts;      /* stripe, inter-frame: width >= 1, offset, stride >= 1 */
     int32_t Sw, So, Ss;      /* stripe, intra-frame: width >= 1, offset, stride >= 1 */
     int32_t layout;          /* vsa_layout: token order of this head (see below)   */
+    int32_t tile_round;      /* 0 exact mask; 1 tile-aligned rounding (see below)  */
 } vsa_mask_spec;
+
+/* tile_round = 1 replaces the head's mask by its tile-aligned rounding, a
+   lossy opt-in mode ("Sparse VideoGen: accelerating video diffusion attention
+   on TPU", "aligning the sparse mask with execution", B3): a tile pair with
+   some kept (real query, real key) pairs is kept whole when at least half of
+   its real pairs are kept and dropped otherwise, so boundary work remains
+   only where a kv tile holds padding slots.  The tile map, the kv-tile lists
+   and the attention follow the rounded mask; vsa_plan_kept_pairs still counts
+   the exact mask.  Allowed for full and SVG spatial / temporal heads
+   (VSA_ERR_UNSUPPORTED otherwise). */
 
 /* Token order of a head inside the [B, heads, n_slots, D] tensors.
    VSA_LAYOUT_TILE_MAJOR: tile-major over the 3D units (bt,bh,bw), padded per

@@ -68,8 +68,13 @@ class GpuRun:
         """Oracle vs GPU on natural query rows of head h; returns (max, mean, lse max)."""
         w = self.w
         rows = np.asarray(rows, dtype=np.int64)
-        o_ref, lse_ref = oracle.attention_rows(w.specs[h], self.grid, w.unit, w.D, w.scale,
-                                               self.q[b, h], self.k[b, h], self.v[b, h], rows)
+        if w.specs[h].get("tile_round", 0):
+            o_ref, lse_ref = oracle.attention_rows_rounded(w.specs[h], self.grid, w.unit, self.plan.n_slots,
+                                                           w.q_tile, w.kv_tile, w.D, w.scale,
+                                                           self.q[b, h], self.k[b, h], self.v[b, h], rows)
+        else:
+            o_ref, lse_ref = oracle.attention_rows(w.specs[h], self.grid, w.unit, w.D, w.scale,
+                                                   self.q[b, h], self.k[b, h], self.v[b, h], rows)
         o_gpu = self.o_rows(b, h, rows)
         lse_gpu = self.lse_natural(b, h)[rows]
         assert np.isfinite(o_gpu).all(), "GPU output has non-finite values"
@@ -93,8 +98,8 @@ class GpuRun:
 
 
 def oracle_map_rows(w: W.Workload, h: int, n_slots: int, qtiles) -> np.ndarray:
-    return oracle.tile_map(w.specs[h], (w.T, w.H, w.W), w.unit, n_slots, w.q_tile, w.kv_tile,
-                           qtiles)
+    fn = oracle.rounded_tile_map if w.specs[h].get("tile_round", 0) else oracle.tile_map
+    return fn(w.specs[h], (w.T, w.H, w.W), w.unit, n_slots, w.q_tile, w.kv_tile, qtiles)
 
 
 def sample_qtiles(n_q: int, k: int, seed: int) -> np.ndarray:

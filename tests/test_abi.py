@@ -67,6 +67,8 @@ def test_plan_create_rejects_bad_arguments_on_host():
         ([W.mask_spec("stripe", Tw=1, Ts=2, Sw=1, Ss=3)], dict(grid=(2, 300, 300), unit=(1, 8, 8)), -2),
         ([dict(ok, layout=1)], dict(), -2),                # frame-0-first order: temporal / full heads only
         ([dict(ok, layout=2)], dict(), -1),                # unknown layout
+        ([dict(W.mask_spec("sta", kt=1, kh=1, kw=1), tile_round=1)], dict(), -2),  # rounding: SVG / full only
+        ([dict(ok, tile_round=2)], dict(), -1),
     ]
     for specs, kw, want in cases:
         rc, handle = _create_raw(specs, **kw)

@@ -9,6 +9,7 @@ rows, and their per-head totals with closed forms where one exists.
 import numpy as np
 import pytest
 
+import oracle
 import workloads as W
 from _helpers import GpuRun, oracle_map_rows, sample_qtiles
 
@@ -98,6 +99,25 @@ def test_svg_wan720p_temporal_frame0_first():
     finally:
         plan.close()
         plan0.close()
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+def test_svg_wan720p_tile_rounded(layout):
+    # the lossy tile-aligned rounding on the full SVG workload: sampled maps
+    # against the oracle's rounded map, sampled rows against attention under
+    # the rounded mask; boundary tiles remain only where a kv tile has padding
+    w = W.svg_wan720p(temporal_layout=layout, tile_round=1)
+    counts, _ = _check(w, [0, 5, 9], 64, [0, 5], qtiles_per_head=6)
+    import block_sparse_attention_mask_b200 as vsa
+    plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile)
+    try:
+        gmap = plan.tile_map()
+        for h in range(w.heads):
+            perm = oracle.tile_major_order((w.T, w.H, w.W), w.unit, plan.n_slots, layout=int(w.specs[h]["layout"]))
+            padded_kv = (perm.reshape(-1, w.kv_tile) < 0).any(axis=1)
+            assert not (gmap[h][:, ~padded_kv] == 1).any()
+    finally:
+        plan.close()
 
 
 def test_sta_hunyuan720p():

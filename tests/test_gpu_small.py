@@ -55,6 +55,15 @@ CASES = {
                             [S("temporal", 1, rh=1, rw=1, layout=1), S("full", 1, layout=1)]),
     "frame0_first_one_frame": ((1, 8, 16), (1, 8, 16), 128, 128, 128,
                                [S("temporal", 0, rh=1, rw=2, layout=1), S("temporal", 1, rh=1, rw=2, layout=1)]),
+    # tile-aligned rounding (lossy mode), next to exact heads
+    "rounded_mixed": ((5, 13, 20), (1, 8, 16), 128, 128, 128,
+                      [S("temporal", 1, rh=2, rw=3, tile_round=1), S("spatial", 1, rt=1, tile_round=1),
+                       S("temporal", 1, rh=1, rw=4, layout=1, tile_round=1), S("full", 0, tile_round=1),
+                       S("temporal", 1, rh=2, rw=3)]),
+    "rounded_q64_k64_d64": ((4, 9, 11), (1, 8, 8), 64, 64, 64,
+                            [S("temporal", 0, rh=1, rw=2, tile_round=1), S("spatial", 0, rt=0, tile_round=1)]),
+    "rounded_token_units": ((3, 7, 9), (1, 1, 1), 128, 64, 64,
+                            [S("temporal", 1, rh=1, rw=1, tile_round=1), S("spatial", 1, rt=0, tile_round=1)]),
 }
 
 
@@ -76,7 +85,8 @@ def test_tile_map_bit_exact(run):
     w = run.w
     gmap = run.plan.tile_map()
     for h in range(w.heads):
-        ref = oracle.tile_map(w.specs[h], run.grid, w.unit, run.plan.n_slots, w.q_tile, w.kv_tile)
+        fn = oracle.rounded_tile_map if w.specs[h].get("tile_round", 0) else oracle.tile_map
+        ref = fn(w.specs[h], run.grid, w.unit, run.plan.n_slots, w.q_tile, w.kv_tile)
         assert (gmap[h] == ref).all(), f"head {h}: {np.argwhere(gmap[h] != ref)[:5]}"
     counts = run.plan.tile_counts()
     for h in range(w.heads):

@@ -113,13 +113,16 @@ def tiny() -> Workload:
                     note="fp32 N(0,1) draw seen by the kernel as bf16")
 
 
-def svg_wan720p(temporal_layout: int = 0) -> Workload:
+def svg_wan720p(temporal_layout: int = 0, tile_round: int = 0) -> Workload:
     """SVG on the Wan 720p latent: 5 spatial + 5 temporal heads with the sink.
     temporal_layout=1 puts the temporal heads in the frame-0-first,
-    position-major order (the temporal-head permutation); same keep sets."""
-    specs = tuple([mask_spec("spatial", sink=1, rt=1)] * 5 +
-                  [mask_spec("temporal", sink=1, rh=5, rw=8, layout=temporal_layout)] * 5)
-    name = "svg_wan720p_21x45x80" + ("_temporal_frame0_first" if temporal_layout else "")
+    position-major order (the temporal-head permutation); same keep sets.
+    tile_round=1 rounds every head's mask to whole tiles (lossy)."""
+    specs = tuple([mask_spec("spatial", sink=1, rt=1, tile_round=tile_round)] * 5 +
+                  [mask_spec("temporal", sink=1, rh=5, rw=8, layout=temporal_layout,
+                             tile_round=tile_round)] * 5)
+    name = ("svg_wan720p_21x45x80" + ("_temporal_frame0_first" if temporal_layout else "") +
+            ("_tile_rounded" if tile_round else ""))
     return Workload(name, 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128, specs)
 
 
@@ -173,7 +176,8 @@ def scaling(T: int, mask: str = "full", q_tile: int = 128, kv_tile: int = 128) -
 
 
 def all_parity_workloads() -> List[Workload]:
-    out = [tiny(), svg_wan720p(), svg_wan720p(temporal_layout=1), sta_hunyuan720p(), stripe_wan720p()]
+    out = [tiny(), svg_wan720p(), svg_wan720p(temporal_layout=1), svg_wan720p(tile_round=1),
+           svg_wan720p(temporal_layout=1, tile_round=1), sta_hunyuan720p(), stripe_wan720p()]
     for T in SCALING_T:
         out.append(scaling(T, "full"))
         out.append(scaling(T, "spatial"))
