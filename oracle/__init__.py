@@ -243,3 +243,42 @@ def attention_rows_rounded(spec, grid, unit, n_slots: int, Bq: int, Bk: int, D: 
         o[i] = (p @ vf[keys]) / p.sum()
         lse[i] = mx + np.log(p.sum())
     return o, lse
+
+
+def svg_route(spatial_specs, temporal_specs, grid, D: int, scale: float,
+              q: np.ndarray, k: np.ndarray, v: np.ndarray, rows,
+              nthreads: Optional[int] = None) -> Tuple[np.ndarray, np.ndarray]:
+    """SVG online profiling: route every head to its spatial or temporal mask.
+
+    "Sparse VideoGen: accelerating video diffusion attention on TPU", section
+    on SVG heads: a few query rows are sampled, their outputs are computed
+    under full attention and under each head's spatial and temporal masks,
+    and the head takes the sparse mask whose outputs deviate least from the
+    full ones (the sample is 1-2% of the tokens, "Video diffusion
+    long-sequence attention and sparsity", section 7).  Readings: the
+    deviation is the mean squared difference over the sampled rows, the batch
+    and the head dimension; a head goes temporal only when its temporal
+    deviation is strictly smaller; the candidates' exact predicates are
+    compared (their token order and rounding switches only change execution).
+
+    q, k, v: bf16 bits [B, Hh, N, D] in natural order; rows: sampled natural
+    token indices, shared by all heads and batches.  Returns (err [Hh, 2]
+    float64 = (spatial, temporal) deviations, flags [Hh] int32, 1 = temporal).
+    """
+    q = np.asarray(q, dtype=np.uint16)
+    B, Hh, N, Dq = q.shape
+    assert Dq == D and N == int(np.prod(grid))
+    rows = np.asarray(rows, dtype=np.int64)
+    full = {f: 0 for f, _ in _Mask._fields_}     # kind 0: every real key kept
+    unit = (1, 1, 1)                              # SVG predicates use no 3D unit
+    err = np.zeros((Hh, 2), dtype=np.float64)
+    for h in range(Hh):
+        for b in range(B):
+            qs, ks, vs = q[b, h], k[b, h], v[b, h]
+            o_full, _ = attention_rows(full, grid, unit, D, scale, qs, ks, vs, rows, nthreads)
+            for c, spec in enumerate((spatial_specs[h], temporal_specs[h])):
+                o_c, _ = attention_rows(spec, grid, unit, D, scale, qs, ks, vs, rows, nthreads)
+                err[h, c] += float(((o_c - o_full) ** 2).sum())
+    err /= float(B * len(rows) * D)
+    flags = (err[:, 1] < err[:, 0]).astype(np.int32)
+    return err, flags

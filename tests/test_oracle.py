@@ -479,3 +479,90 @@ def test_rounded_attention_against_dense_reference():
     o_ref = (p @ vf) / p.sum(axis=1, keepdims=True)
     o, _ = oracle.attention_rows_rounded(spec, grid, unit, 128, B, B, D, w.scale, q, k, v, np.arange(N))
     assert np.abs(o - o_ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# SVG routing (sampled-query profiling of spatial vs temporal masks)
+
+
+def _route(sp, tm, grid, D, q, k, v, rows, scale=None):
+    scale = scale if scale is not None else 1.0 / np.sqrt(D)
+    return oracle.svg_route(sp, tm, grid, D, scale, q, k, v, rows)
+
+
+def _rand_bits(shape, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    return W.bf16_bits_from_f32(g.standard_normal(shape, dtype=np.float32))
+
+
+def test_route_uniform_weights_closed_form():
+    # q = 0 makes every kept key weigh the same, so each output is the mean of
+    # v over the kept keys.  Grid T=3, H=2, W=3 (token n = (t*2 + h)*3 + w).
+    # Row 17 = (t2, h1, w2): spatial rt=0 + sink keeps frames 0 and 2 = tokens
+    # 0..5, 12..17; temporal rh=0, rw=1 keeps h=1, w in {1,2} of every frame =
+    # tokens 4,5,10,11,16,17.  Row 0 = (t0, h0, w0): spatial keeps frame 0 =
+    # 0..5; temporal keeps h=0, w in {0,1} = 0,1,6,7,12,13.
+    grid, D = (3, 2, 3), 4
+    q = np.zeros((1, 1, 18, D), dtype=np.uint16)
+    k = _rand_bits((1, 1, 18, D), 1)
+    v = _rand_bits((1, 1, 18, D), 2)
+    vf = W.bf16_bits_to_f32(v[0, 0]).astype(np.float64)
+    sp = [W.mask_spec("spatial", sink=1, rt=0)]
+    tm = [W.mask_spec("temporal", sink=0, rh=0, rw=1)]
+    err, flags = _route(sp, tm, grid, D, q, k, v, [0, 17])
+    full = vf.mean(axis=0)
+    keep = {(17, 0): list(range(6)) + list(range(12, 18)), (17, 1): [4, 5, 10, 11, 16, 17],
+            (0, 0): list(range(6)), (0, 1): [0, 1, 6, 7, 12, 13]}
+    for c in (0, 1):
+        want = sum(((vf[keep[(r, c)]].mean(axis=0) - full) ** 2).sum() for r in (0, 17)) / (2 * D)
+        assert err[0, c] == pytest.approx(want, rel=1e-12, abs=1e-300)
+    assert flags[0] == int(err[0, 1] < err[0, 0])
+
+
+def test_route_keep_all_candidate_has_zero_deviation():
+    grid, D = (4, 3, 5), 8
+    N = 60
+    q, k, v = (_rand_bits((2, 2, N, D), s) for s in (3, 4, 5))
+    rows = [0, 7, 33, 59]
+    # head 0: the spatial candidate keeps every key; head 1: the temporal one
+    sp = [W.mask_spec("spatial", sink=0, rt=3), W.mask_spec("spatial", sink=0, rt=0)]
+    tm = [W.mask_spec("temporal", sink=1, rh=0, rw=0), W.mask_spec("temporal", sink=0, rh=2, rw=4)]
+    err, flags = _route(sp, tm, grid, D, q, k, v, rows)
+    assert err[0, 0] == 0.0 and err[0, 1] > 0.0 and flags[0] == 0
+    assert err[1, 1] == 0.0 and err[1, 0] > 0.0 and flags[1] == 1
+
+
+def test_route_tie_goes_spatial_and_batches_average():
+    grid, D = (3, 4, 4), 8
+    N = 48
+    q, k, v = (_rand_bits((2, 1, N, D), s) for s in (6, 7, 8))
+    rows = [1, 20, 47]
+    same = W.mask_spec("spatial", sink=1, rt=0)
+    err, flags = _route([same], [same], grid, D, q, k, v, rows)
+    assert err[0, 0] == err[0, 1] > 0.0 and flags[0] == 0
+    # the deviation is a mean over the batch: the two batches' own deviations
+    tm = W.mask_spec("temporal", sink=1, rh=1, rw=1)
+    e2, _ = _route([same], [tm], grid, D, q, k, v, rows)
+    e0, _ = _route([same], [tm], grid, D, q[:1], k[:1], v[:1], rows)
+    e1, _ = _route([same], [tm], grid, D, q[1:], k[1:], v[1:], rows)
+    np.testing.assert_allclose(e2, (e0 + e1) / 2, rtol=1e-12)
+
+
+def test_route_picks_the_pattern_the_heads_follow():
+    # frame-structured q/k attend within their frame (the pages' spatial
+    # heads), position-structured ones to their position across frames (the
+    # temporal heads)
+    w = W.tiny_routing()
+    q, k, v = (W.full_tensor(w, x) for x in "qkv")
+    rows = W.route_rows(w.N, 0.05)
+    sp = [a for a, _ in w.route_specs]
+    tm = [b for _, b in w.route_specs]
+    err, flags = _route(sp, tm, (w.T, w.H, w.W), w.D, q, k, v, rows)
+    assert flags[0] == 0 and flags[1] == 1 and flags[3] == 0
+    assert err[0, 0] < 1e-3 * err[0, 1] and err[1, 1] < 1e-3 * err[1, 0]
+
+
+def test_route_rows_sample():
+    r = W.route_rows(75600, 0.01)
+    assert len(r) == 756 and len(np.unique(r)) == 756 and r.min() >= 0 and r.max() < 75600
+    assert np.all(np.diff(r) > 0)

@@ -85,6 +85,12 @@ class Workload:
     specs: Tuple[Dict[str, int], ...]
     seeds: Tuple[int, int, int] = (0, 1, 2)
     note: str = ""
+    # per-head structure of the q/k draws: "" iid, "frame" or "position" (see
+    # ``head_tensor``); empty tuple = iid everywhere
+    structure: Tuple[str, ...] = ()
+    structure_amp: float = 0.0
+    # candidate masks for SVG routing (one pair per head), empty if not routed
+    route_specs: Tuple[Tuple[Dict[str, int], Dict[str, int]], ...] = ()
 
     @property
     def N(self) -> int:
@@ -124,6 +130,30 @@ def svg_wan720p(temporal_layout: int = 0, tile_round: int = 0) -> Workload:
     name = ("svg_wan720p_21x45x80" + ("_temporal_frame0_first" if temporal_layout else "") +
             ("_tile_rounded" if tile_round else ""))
     return Workload(name, 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128, specs)
+
+
+def svg_wan720p_routing(amp: float = 10.0) -> Workload:
+    """SVG routing on the Wan 720p latent: every head has both candidates
+    (spatial |dt| <= 1 and temporal |dh| <= 5, |dw| <= 8, both with the
+    frame-0 sink).  The q/k draws of heads 0-4 carry a per-frame embedding and
+    those of heads 5-9 a per-position embedding, so that the former attend
+    within their frame (spatial heads) and the latter to their position across
+    frames (temporal heads).  The plan starts with every head spatial."""
+    sp = mask_spec("spatial", sink=1, rt=1)
+    tm = mask_spec("temporal", sink=1, rh=5, rw=8)
+    return Workload("svg_wan720p_routing_21x45x80", 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128,
+                    tuple([sp] * 10), structure=tuple(["frame"] * 5 + ["position"] * 5),
+                    structure_amp=amp, route_specs=tuple([(sp, tm)] * 10))
+
+
+def tiny_routing(amp: float = 10.0) -> Workload:
+    """4x8x8 grid, 4 heads (frame, position, iid, frame structure), d=64,
+    candidates spatial |dt| <= 1 and temporal |dh|, |dw| <= 1, with the sink."""
+    sp = mask_spec("spatial", sink=1, rt=1)
+    tm = mask_spec("temporal", sink=1, rh=1, rw=1)
+    return Workload("tiny_routing_4x8x8", 2, 4, 8, 8, 4, 64, (1, 8, 8), 64, 64, tuple([sp] * 4),
+                    structure=("frame", "position", "", "frame"), structure_amp=amp,
+                    route_specs=tuple([(sp, tm)] * 4))
 
 
 def sta_hunyuan720p() -> Workload:
@@ -209,10 +239,36 @@ def head_draw_f32(seed: int, b: int, h: int, n: int, d: int) -> np.ndarray:
     return g.standard_normal(n * d, dtype=np.float32).reshape(n, d)
 
 
+def structure_embedding(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray]:
+    """(class index of every natural token [N], unit-norm embeddings [C, D])
+    of head ``h``: class = frame t for "frame", (h, w) position for
+    "position".  Drawn from ``PCG64(SeedSequence([seeds[0] + 1000, h]))``."""
+    kind = w.structure[h]
+    n = np.arange(w.N)
+    if kind == "frame":
+        cls, C = n // (w.H * w.W), w.T
+    elif kind == "position":
+        cls, C = n % (w.H * w.W), w.H * w.W
+    else:
+        raise ValueError(f"no structure for head {h}")
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seeds[0] + 1000, h])))
+    e = g.standard_normal((C, w.D))
+    e /= np.linalg.norm(e, axis=1, keepdims=True)
+    return cls, e.astype(np.float32)
+
+
 def head_tensor(w: Workload, which: str, b: int, h: int) -> np.ndarray:
-    """bf16 bits [N, D] of tensor ``which`` for batch ``b``, head ``h`` (natural order)."""
+    """bf16 bits [N, D] of tensor ``which`` for batch ``b``, head ``h`` (natural order).
+
+    With a structured head, q and k both get ``structure_amp`` times the
+    head's embedding of each token's class added to the N(0,1) draw before
+    the bf16 rounding; v stays iid."""
     seed = w.seeds["qkv".index(which)]
-    return bf16_bits_from_f32(head_draw_f32(seed, b, h, w.N, w.D))
+    x = head_draw_f32(seed, b, h, w.N, w.D)
+    if which in "qk" and w.structure and w.structure[h]:
+        cls, e = structure_embedding(w, h)
+        x += np.float32(w.structure_amp) * e[cls]
+    return bf16_bits_from_f32(x)
 
 
 def full_tensor(w: Workload, which: str, heads: Optional[Sequence[int]] = None,
@@ -241,6 +297,14 @@ def full_tensor(w: Workload, which: str, heads: Optional[Sequence[int]] = None,
         with ThreadPoolExecutor(n) as ex:
             list(ex.map(fill, jobs))
     return out
+
+
+def route_rows(N: int, frac: float = 0.01, seed: int = 11) -> np.ndarray:
+    """The query sample of SVG routing: round(frac * N) (at least 1) distinct
+    natural token indices drawn uniformly from ``PCG64(seed)``, ascending."""
+    R = max(1, int(round(frac * N)))
+    g = np.random.Generator(np.random.PCG64(seed))
+    return np.sort(g.choice(N, size=min(R, N), replace=False)).astype(np.int64)
 
 
 def sample_rows(w: Workload, head: int, R: int, seed: int = 7) -> np.ndarray:
