@@ -41,13 +41,16 @@ import workloads as W  # noqa: E402
 METRIC = "sparse attn fwd ms & effective TFLOPS (kept tiles) vs B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # kernels launched per ABI call (claimed launch count inside the timed region)
-LAUNCHES = {"plan_build": 3, "plan_build_stripe": 4, "permute": 1, "unpermute": 1, "fwd": 1}
+LAUNCHES = {"plan_build": 3, "plan_build_stripe": 4, "permute": 1, "unpermute": 1, "fwd": 1,
+            "route": 3, "apply": 1}
+ROUTE_FRAC = 0.01      # sampled share of the tokens for SVG routing
 
 WORKLOADS = {
     "svg_wan720p": W.svg_wan720p,
     "svg_wan720p_temporal_f0": lambda: W.svg_wan720p(temporal_layout=1),
     "svg_wan720p_rounded": lambda: W.svg_wan720p(tile_round=1),
     "svg_wan720p_temporal_f0_rounded": lambda: W.svg_wan720p(temporal_layout=1, tile_round=1),
+    "svg_wan720p_routing": W.svg_wan720p_routing,
     "tiny": W.tiny,
     "sta_hunyuan720p": W.sta_hunyuan720p,
     "stripe_wan720p": W.stripe_wan720p,
@@ -141,8 +144,8 @@ def exec_flops(w, counts) -> float:
 def rank_workload(w, rank: int):
     """The workload rank `rank` processes: same shape and masks, its own batch
     element (independent seeds), so per-GPU work is fixed as ranks are added."""
-    return W.Workload(w.name, w.B, w.T, w.H, w.W, w.heads, w.D, w.unit, w.q_tile, w.kv_tile,
-                      w.specs, seeds=tuple(s + 1000 * rank for s in w.seeds))
+    from dataclasses import replace
+    return replace(w, seeds=tuple(s + 1000 * rank for s in w.seeds))
 
 
 def aggregate_tflops(flops_per_rank_step: float, world: int, ms_max: float) -> float:
@@ -293,10 +296,41 @@ def run_gpu(args, w, world, rank, local):
     per_step_launches = (LAUNCHES["plan_build_stripe"] if has_stripe else LAUNCHES["plan_build"]) \
         + 3 * LAUNCHES["permute"] + LAUNCHES["fwd"] + LAUNCHES["unpermute"]
 
+    # SVG routing before the plan build: sampled-query profiling, then the
+    # per-head switch (which rebuilds the plan on the device)
+    routed = bool(w.route_specs)
+    route_events = []
+    if routed:
+        plan.set_route_candidates([a for a, _ in w.route_specs], [b for _, b in w.route_specs], stream)
+        rows_np = W.route_rows(w.N, ROUTE_FRAC).astype(np.int32)
+        with torch.cuda.stream(stream):
+            rows_d = torch.from_numpy(rows_np).to(dev)
+            ws = torch.empty(vsa.vsa_svg_route_workspace_size(h, B, w.D, len(rows_np)),
+                             dtype=torch.uint8, device=dev)
+            r_err = torch.empty((w.heads, 2), dtype=torch.float32, device=dev)
+            r_flags = torch.empty((w.heads,), dtype=torch.int32, device=dev)
+        stream.synchronize()
+        per_step_launches += LAUNCHES["route"] + LAUNCHES["apply"]
+
+    def plan_step(qn, kn, vn, record: bool):
+        if not routed:
+            vsa.vsa_plan_build(h, sh)
+            return
+        if record:
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+        vsa.vsa_svg_route(h, qn, kn, vn, B, w.D, rows_d, len(rows_np), w.scale, r_err, r_flags, ws,
+                          ws.numel(), sh)
+        if record:
+            e1.record(stream)
+            route_events.append((e0, e1))
+        vsa.vsa_plan_apply_route(h, r_flags, sh)
+
     fwd_events = []
 
     def step(record_fwd: bool):
-        vsa.vsa_plan_build(h, sh)
+        plan_step(q, k, v, record_fwd)
         vsa.vsa_permute(h, q, qp, B, w.D, sh)
         vsa.vsa_permute(h, k, kp, B, w.D, sh)
         vsa.vsa_permute(h, v, vp, B, w.D, sh)
@@ -345,6 +379,8 @@ def run_gpu(args, w, world, rank, local):
     plan.check(stream)
     ms_steps = [a.elapsed_time(b) for a, b in step_events]
     ms_fwd = [a.elapsed_time(b) for a, b in fwd_events]
+    ms_route = max_over_ranks(statistics.mean([a.elapsed_time(b) for a, b in route_events]), world, dev) \
+        if routed else None
     ms_step = max_over_ranks(statistics.mean(ms_steps), world, dev)
     ms_fwd_mean = max_over_ranks(statistics.mean(ms_fwd), world, dev)
     value = aggregate_tflops(flops_step, world, ms_step)
@@ -358,7 +394,7 @@ def run_gpu(args, w, world, rank, local):
         qd.copy_(pinned[0], non_blocking=True)
         kd.copy_(pinned[1], non_blocking=True)
         vd.copy_(pinned[2], non_blocking=True)
-        vsa.vsa_plan_build(h, sh)
+        plan_step(qd, kd, vd, False)
         vsa.vsa_permute(h, qd, qp, B, w.D, sh)
         vsa.vsa_permute(h, kd, kp, B, w.D, sh)
         vsa.vsa_permute(h, vd, vp, B, w.D, sh)
@@ -435,6 +471,12 @@ def run_gpu(args, w, world, rank, local):
                       "boundary_share_of_executed": float(counts[:, 1].sum() / max(1, counts[:, 1:].sum()))},
             "exec_steps": int(steps_exec.sum()),
             "cpu_baseline": cpu,
+            "route": None if not routed else {
+                "ms": ms_route, "rows": int(len(rows_np)),
+                "flags": [int(x) for x in r_flags.cpu().numpy()],
+                # four R x N x D products (QK^T and three PV) over the sampled rows
+                "tflops": 8.0 * B * w.heads * len(rows_np) * w.N * w.D / (ms_route * 1e-3) / 1e12,
+                "frac": 8.0 * B * w.heads * len(rows_np) * w.N * w.D / (ms_route * 1e-3) / 1e12 / peak},
             "e2e": {"value": aggregate_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
                     "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "clocks": clk,
@@ -448,13 +490,15 @@ _REV = None
 
 
 def kernel_rev() -> str:
-    """Hash of the attention kernel source, to tie stored ncu counters to it."""
+    """Hash of the attention kernel's sources, to tie stored ncu counters to them."""
     global _REV
     if _REV is None:
         import hashlib
-        p = os.path.join(ROOT, "block_sparse_attention_mask_b200", "csrc", "vsa_attn.cu")
-        with open(p, "rb") as f:
-            _REV = hashlib.sha256(f.read()).hexdigest()[:16]
+        h = hashlib.sha256()
+        for f in ("vsa_attn.cu", "vsa_sm100.cuh"):
+            with open(os.path.join(ROOT, "block_sparse_attention_mask_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+        _REV = h.hexdigest()[:16]
     return _REV
 
 

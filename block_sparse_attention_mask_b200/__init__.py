@@ -81,6 +81,10 @@ def _load() -> ctypes.CDLL:
         "vsa_selftest_watchdog": ([vp, ctypes.c_longlong, vp], i32),
         "vsa_tile_map_noalloc": ([P(vsa_mask_spec), i32, i32, i32, i32, i32, i32, i32, i32, i32, vp,
                                   sz, vp], i32),
+        "vsa_plan_set_route_candidates": ([vp, P(vsa_mask_spec), P(vsa_mask_spec), vp], i32),
+        "vsa_svg_route_workspace_size": ([vp, i32, i32, i32, P(sz)], i32),
+        "vsa_svg_route": ([vp, vp, vp, vp, i32, i32, vp, i32, f32, vp, vp, vp, sz, vp], i32),
+        "vsa_plan_apply_route": ([vp, vp, vp], i32),
         "vsa_status_string": ([i32], ctypes.c_char_p),
         "vsa_version": ([], i32),
     }
@@ -256,6 +260,35 @@ def vsa_version() -> int:
     return int(_lib.vsa_version())
 
 
+def vsa_plan_set_route_candidates(plan: int, spatial: Sequence[Dict[str, int]],
+                                  temporal: Sequence[Dict[str, int]], stream=None) -> None:
+    n = len(spatial)
+    if len(temporal) != n:
+        raise ValueError("one spatial and one temporal candidate per head")
+    sa = (vsa_mask_spec * n)(*[make_spec(d) for d in spatial])
+    ta = (vsa_mask_spec * n)(*[make_spec(d) for d in temporal])
+    _check(_lib.vsa_plan_set_route_candidates(plan, sa, ta, _stream(stream)),
+           "vsa_plan_set_route_candidates")
+
+
+def vsa_svg_route_workspace_size(plan: int, B: int, D: int, n_rows: int) -> int:
+    out = ctypes.c_size_t(0)
+    _check(_lib.vsa_svg_route_workspace_size(plan, B, D, n_rows, ctypes.byref(out)),
+           "vsa_svg_route_workspace_size")
+    return int(out.value)
+
+
+def vsa_svg_route(plan: int, q, k, v, B: int, D: int, rows, n_rows: int, scale: float, err, flags,
+                  workspace, workspace_bytes: int, stream=None) -> None:
+    _check(_lib.vsa_svg_route(plan, _ptr(q), _ptr(k), _ptr(v), B, D, _ptr(rows), n_rows, scale,
+                              _ptr(err), _ptr(flags), _ptr(workspace), workspace_bytes,
+                              _stream(stream)), "vsa_svg_route")
+
+
+def vsa_plan_apply_route(plan: int, flags, stream=None) -> None:
+    _check(_lib.vsa_plan_apply_route(plan, _ptr(flags), _stream(stream)), "vsa_plan_apply_route")
+
+
 # ---------------------------------------------------------------------------
 # convenience wrapper
 
@@ -302,6 +335,15 @@ class Plan:
 
     def check(self, stream=None) -> None:
         vsa_check_status(self.handle, stream)
+
+    def set_route_candidates(self, spatial: Sequence[Dict[str, int]],
+                             temporal: Sequence[Dict[str, int]], stream=None) -> None:
+        vsa_plan_set_route_candidates(self.handle, spatial, temporal, stream)
+
+    def apply_route(self, flags, stream=None) -> None:
+        """Switch every head to its temporal (flag 1) or spatial candidate and
+        rebuild the maps on the device; ``flags`` is a device int32 [heads]."""
+        vsa_plan_apply_route(self.handle, flags, stream)
 
 
 def _require_bf16(t, shape: Tuple[int, ...], name: str) -> None:
@@ -360,3 +402,33 @@ def attention(plan: Plan, q, k, v, scale: Optional[float] = None, stream=None):
     vp = permute(plan, v, stream=stream)
     op, lse = sparse_attn_fwd(plan, qp, kp, vp, scale, stream=stream)
     return unpermute(plan, op, stream=stream), lse
+
+
+def svg_route(plan: Plan, q, k, v, rows, scale: Optional[float] = None, workspace=None,
+              err=None, flags=None, stream=None):
+    """Sampled-query routing of every head (natural-order q, k, v [B, Hh, N, D]
+    bf16; rows: device int32 [R] natural token indices).  Returns (err fp32
+    [Hh, 2] spatial / temporal deviations, flags int32 [Hh], 1 = temporal),
+    both on the device; nothing synchronises."""
+    import torch
+    B, Hh, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16(t, (B, plan.heads, plan.n_tokens, D), name)
+    if rows.dtype != torch.int32 or not rows.is_cuda or not rows.is_contiguous() or rows.dim() != 1:
+        raise ValueError("rows must be a contiguous int32 CUDA vector")
+    R = int(rows.shape[0])
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    need = vsa_svg_route_workspace_size(plan.handle, B, D, R)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    if workspace.numel() * workspace.element_size() < need:
+        raise ValueError(f"workspace needs {need} bytes")
+    if err is None:
+        err = torch.empty((Hh, 2), dtype=torch.float32, device=q.device)
+    if flags is None:
+        flags = torch.empty((Hh,), dtype=torch.int32, device=q.device)
+    vsa_svg_route(plan.handle, q, k, v, B, D, rows, R, scale, err, flags, workspace,
+                  workspace.numel() * workspace.element_size(), stream)
+    return err, flags
+

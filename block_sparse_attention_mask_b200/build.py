@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libvsa.so")
-SOURCES = ["vsa_plan.cu", "vsa_permute.cu", "vsa_attn.cu", "vsa_api.cu", "vsa_noalloc.cu"]
+SOURCES = ["vsa_plan.cu", "vsa_permute.cu", "vsa_attn.cu", "vsa_route.cu", "vsa_api.cu", "vsa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -26,7 +26,8 @@ def nvcc() -> str:
 
 def _inputs() -> List[str]:
     files = [os.path.join(CSRC, s) for s in SOURCES]
-    files += [os.path.join(CSRC, "vsa_internal.h"), os.path.join(INCLUDE, "vsa.h")]
+    files += [os.path.join(CSRC, f) for f in sorted(os.listdir(CSRC)) if f.endswith((".h", ".cuh"))]
+    files += [os.path.join(INCLUDE, "vsa.h")]
     return files
 
 
@@ -46,12 +47,13 @@ def build(force: bool = False, verbose: bool = False, extra: List[str] | None = 
              "--expt-relaxed-constexpr"] + ARCH + (extra or [])
     if verbose:
         flags += ["-Xptxas", "-v"]
-    objs = []
-    for src in SOURCES:
-        obj = os.path.join(objdir, src.replace(".cu", ".o"))
-        cmd = [nvcc(), "-c", os.path.join(CSRC, src), "-o", obj] + flags
-        subprocess.check_call(cmd)
-        objs.append(obj)
+    objs = [os.path.join(objdir, src.replace(".cu", ".o")) for src in SOURCES]
+    cmds = [[nvcc(), "-c", os.path.join(CSRC, src), "-o", obj] + flags for src, obj in zip(SOURCES, objs)]
+    # translation units compile in parallel
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+        for _ in ex.map(subprocess.check_call, cmds):
+            pass
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), "-shared", "-o", tmp] + objs + ARCH + ["-cudart", "static"])
     os.replace(tmp, LIB)

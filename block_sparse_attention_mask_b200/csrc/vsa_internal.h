@@ -49,6 +49,8 @@ struct vsa_plan_s {
     unsigned long long* d_steps;   // [heads] executed steps
     unsigned int* d_status;     // watchdog / state flags
     int has_stripe;
+    vsa_mask_spec* d_cand;      // [2][heads] SVG routing candidates: spatial, temporal
+    int has_cand;
 };
 
 // Host helpers ------------------------------------------------------------

@@ -581,6 +581,7 @@ static void free_plan(vsa_plan_s* p)
     cudaFree(p->d_counts);
     cudaFree(p->d_steps);
     cudaFree(p->d_status);
+    cudaFree(p->d_cand);
     delete p;
 }
 

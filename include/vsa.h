@@ -11,6 +11,8 @@
  *   vsa_permute       q, k, v  natural [B,Hh,N,D] -> tile-major [B,Hh,n_slots,D]
  *   vsa_sparse_attn_fwd       tile-major q,k,v -> tile-major o, lse
  *   vsa_unpermute     o  tile-major -> natural [B,Hh,N,D]
+ *   vsa_svg_route     sampled-query profiling -> per-head spatial / temporal
+ *                     flags; vsa_plan_apply_route switches the heads' specs
  *
  * Sources (web pages on block-sparse video attention):
  *  [SVG-TPU] "Sparse VideoGen: accelerating video diffusion attention on TPU"
@@ -251,6 +253,51 @@ int vsa_unpermute(vsa_plan_t plan, const void* in, void* out, int B, int D, void
 int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v,
                         void* o, float* lse, vsa_plan_t plan,
                         int B, int D, float scale, void* stream);
+
+/* ---- SVG routing: spatial or temporal mask per head ----------------------
+ * [SVG-TPU] section on SVG heads: a few query rows are sampled, their outputs
+ * are computed under full attention and under each head's spatial and
+ * temporal masks, and the head takes the mask whose outputs deviate least
+ * from the full ones ([VDS]: the sample is 1-2% of the tokens).  [SVG-TPU]
+ * "supporting dynamic routing with fixed tensor shapes": the per-head flags
+ * select the candidate spec, and with it the head's token order, without
+ * changing any tensor shape, so the steps after routing run unchanged.
+ *
+ * vsa_plan_set_route_candidates: the two candidates of every head (host
+ * arrays of num_heads specs, copied before return; spatial[h].kind must be
+ * VSA_MASK_SVG_SPATIAL and temporal[h].kind VSA_MASK_SVG_TEMPORAL, each
+ * valid for vsa_plan_create, else VSA_ERR_INVALID_ARG / _UNSUPPORTED).  Their
+ * layout and tile_round fields only take effect once applied; routing
+ * compares the exact predicates.  Synchronises `stream`. */
+int vsa_plan_set_route_candidates(vsa_plan_t plan, const vsa_mask_spec* spatial,
+                                  const vsa_mask_spec* temporal, void* stream);
+
+/* Bytes of device workspace vsa_svg_route needs for B batches, head dim D
+ * and n_rows sampled rows on the current device. */
+int vsa_svg_route_workspace_size(vsa_plan_t plan, int B, int D, int n_rows, size_t* bytes);
+
+/* Deviation of each candidate from full attention over sampled rows.
+ * q, k, v: bf16 [B][num_heads][N][D] in natural (t, h, w) order (device,
+ * 16-byte aligned); rows: device int32 [n_rows] natural token indices shared
+ * by every (batch, head) (an index outside [0, N) is read as 0 and flags
+ * VSA_ERR_DEVICE in vsa_check_status).  Outputs (device): err fp32
+ * [num_heads][2] = mean over batch, rows and D of (o_spatial - o_full)^2 and
+ * (o_temporal - o_full)^2; flags int32 [num_heads] = 1 iff the temporal
+ * deviation is strictly smaller.  workspace: device, 16-byte aligned, at
+ * least vsa_svg_route_workspace_size bytes, owned by the caller.  Needs
+ * candidates (VSA_ERR_INVALID_ARG otherwise).  D in {64,128}.  Asynchronous;
+ * no host synchronisation, capturable in a CUDA graph. */
+int vsa_svg_route(vsa_plan_t plan, const void* q, const void* k, const void* v,
+                  int B, int D, const int32_t* rows, int n_rows, float scale,
+                  float* err, int32_t* flags, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Applies device flags [num_heads] (nonzero = temporal): each head's spec
+ * becomes its temporal or spatial candidate, then the tile map, the
+ * per-query-block lists and the counts are rebuilt on the device.  Shapes
+ * (n_slots, list capacity) are unchanged; vsa_permute / vsa_unpermute pick
+ * each head's token order from the new specs.  Asynchronous, capturable. */
+int vsa_plan_apply_route(vsa_plan_t plan, const int32_t* flags, void* stream);
 
 /* Synchronises `stream`, then reports and clears the plan's device status
  * word: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_DEVICE; VSA_ERR_CUDA if the

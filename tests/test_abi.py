@@ -91,6 +91,11 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_sparse_attn_fwd(None, None, None, None, None, None, 1, 128, 0.1, None) == -1
     assert L.vsa_check_status(None, None) == -1
     assert L.vsa_selftest_watchdog(None, 1000, None) == -1
+    assert L.vsa_plan_set_route_candidates(None, None, None, None) == -1
+    n = ctypes.c_size_t(0)
+    assert L.vsa_svg_route_workspace_size(None, 1, 128, 1, ctypes.byref(n)) == -1
+    assert L.vsa_svg_route(None, None, None, None, 1, 128, None, 1, 0.1, None, None, None, 0, None) == -1
+    assert L.vsa_plan_apply_route(None, None, None) == -1
 
 
 def test_layout_slot_counts():
