@@ -14,27 +14,36 @@
 // with fixed tensor shapes").
 //
 // route_partial_kernel: one CTA = 128 sampled rows of one (batch, head) and a
-// contiguous range of kv tiles (128 natural keys each; the key range of a
-// head is split across CTAs so that the grid fills the SMs).  8 warps:
-//   warps 4..7  gather the 128 sampled q rows into shared memory (128-byte
+// contiguous range of kv tiles (64 natural keys each; the key range of a
+// head is split across CTAs so that the grid fills the SMs).  12 warps:
+//   warps 8..11 gather the 128 sampled q rows into shared memory (128-byte
 //               swizzled, K-major), then
-//   warp 4      TMA producer: lane 0 K tiles, lane 1 V tiles, 2-stage rings;
-//   warp 5      MMA issuer (one elected lane): S = Q K^T into TMEM (both
-//               operands in shared memory); then O_full += P_full V and
-//               O_sp += P_sp V with P read from TMEM (P_full over the first
-//               64 columns of S, P_sp over the next 64), O_tm += P_tm V with
-//               P_tm in shared memory.  The next tile's S is queued behind
-//               the three PV MMAs, so P is read before S is overwritten.
-//   warps 0..3  softmax: thread r owns sampled row r.  One running max (of
-//               the full row) serves all three accumulators: p = 2^(s*scale*
-//               log2e - m) once per key, masked by the spatial and temporal
-//               keep bits into P_sp and P_tm; three running sums.
-// TMEM: S [0,128), O_full [128,128+D), O_sp, O_tm after it: 512 columns for
-// D = 128.  Each CTA writes its partial (max, three sums, three unnormalised
-// outputs); route_combine_kernel merges the partials of a row, normalises,
-// and forms the row's squared deviations; route_reduce_kernel sums them per
-// head in a fixed order (deterministic) and sets the flag.
-// Every mbarrier wait is bounded (VSA_DEV_TIMEOUT in the status word).
+//   warp 8      TMA producer: lane 0 K tiles, lane 1 V tiles (3-stage rings);
+//   warp 9      MMA issuer (one elected lane): S_j = Q K_j^T into S_{j mod 2}
+//               (both operands in shared memory), then O_full += P_full V_j
+//               and O_sp += P_sp V_j with P read from TMEM (P_full over
+//               columns [0, 32) of S_{j mod 2}, P_sp over [32, 64)) and
+//               O_tm += P_tm V_j with P_tm in shared memory (two buffers).
+//               Issue order QK_0, QK_1, PV_0, QK_2, PV_1, ...: S_{j+2} is
+//               queued behind PV_j, so P_j is read before it is overwritten,
+//               and QK_{j+1} runs while the softmax works on tile j.
+//   warps 0..7  softmax: thread r of warpgroup G owns sampled row r and keys
+//               [32G, 32G + 32) of every tile.  The two warpgroups exchange
+//               their partial row maxima through shared memory, so both keep
+//               the same running max; one running max (of the full row)
+//               serves all three accumulators: p = 2^(s*scale*log2e - m) once
+//               per key, masked by the spatial and temporal keep bits into
+//               P_sp and P_tm; three running sums per warpgroup.
+// The three accumulators are shared by consecutive tiles, so a rescale (when
+// the running max grows by more than 2^8) first waits for the previous
+// tile's PV MMAs.
+// TMEM: S_0 [0,64), S_1 [64,128), O_full [128,128+D), O_sp, O_tm after it:
+// 512 columns for D = 128.  Each CTA writes its partial (max, three sums,
+// three unnormalised outputs); route_combine_kernel merges the partials of a
+// row, normalises, and forms the row's squared deviations;
+// route_reduce_kernel sums them per head in a fixed order (deterministic)
+// and sets the flag.  Every mbarrier wait is bounded (VSA_DEV_TIMEOUT in the
+// status word).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -47,10 +56,11 @@
 namespace {
 
 constexpr int kRRows = 128;                 // sampled rows per CTA (TMEM lanes)
-constexpr int kRBK = 128;                   // keys per kv tile
-constexpr int kRThreads = 256;
-constexpr int kRProducerWarp = 4;
-constexpr int kRMmaWarp = 5;
+constexpr int kRBK = 64;                    // keys per kv tile
+constexpr int kRSoftmaxWarps = 8;           // two warpgroups, 32 keys of a tile each
+constexpr int kRProducerWarp = 8;
+constexpr int kRMmaWarp = 9;
+constexpr int kRThreads = 384;
 constexpr float kRRescale = 8.0f;           // lazy rescale threshold, log2 units
 constexpr int kRMaxSplits = 64;
 constexpr int kRDChunk = 16;                // output columns per combine CTA
@@ -58,26 +68,28 @@ constexpr int kRDChunk = 16;                // output columns per combine CTA
 template <int D>
 struct RCfg {
     static constexpr int Q_BYTES = kRRows * D * 2;
-    static constexpr int P_BYTES = kRRows * kRBK * 2;
+    static constexpr int P_BYTES = kRRows * kRBK * 2;      // one P_tm buffer (one 64-key block)
     static constexpr int KV_BYTES = kRBK * D * 2;
-    static constexpr int STAGES = 2;
+    static constexpr int STAGES = 3;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_P = OFF_Q + Q_BYTES;
-    static constexpr int OFF_K = OFF_P + P_BYTES;
+    static constexpr int OFF_P = OFF_Q + Q_BYTES;           // two P_tm buffers
+    static constexpr int OFF_K = OFF_P + 2 * P_BYTES;
     static constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-    static constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
-    // k_full[2], k_empty[2], v_full[2], v_empty[2], q_full, s_full, p_full, pv_done, drain
-    static constexpr int NBAR = 4 * STAGES + 5;
+    // the two warpgroups' running sums for the epilogue [2][3][128]
+    static constexpr int OFF_SUM = OFF_V + STAGES * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_SUM + 2 * 3 * kRRows * 4;
+    // k_full[3], k_empty[3], v_full[3], v_empty[3], q_full, s_full[2], p_full[2], pv_done, drain,
+    // all_done, s_read[2]
+    static constexpr int NBAR = 4 * STAGES + 10;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;   // tmem addr, abort, issued[3]
     static constexpr int SMEM = OFF_MISC + 20;
-    static constexpr int COL_S = 0;
-    static constexpr int COL_OF = kRBK;
-    static constexpr int COL_OS = kRBK + D;
-    static constexpr int COL_OT = kRBK + 2 * D;
+    static constexpr int COL_S0 = 0;
+    static constexpr int COL_S1 = kRBK;
+    static constexpr int COL_OF = 2 * kRBK;
     static constexpr int TMEM_COLS = 512;
-    static_assert(kRBK + 3 * D <= TMEM_COLS, "TMEM budget");
+    static_assert(2 * kRBK + 3 * D <= TMEM_COLS, "TMEM budget");
     // kind::f16 instruction descriptors: D f32, A/B bf16, M = 128;
-    // QK: A and B K-major, N = 128; PV: B MN-major, N = D
+    // QK: A and B K-major, N = 64; PV: B MN-major, N = D
     static constexpr uint32_t IDESC_QK = (1u << 4) | (1u << 7) | (1u << 10) |
                                          ((uint32_t)(kRBK >> 3) << 17) | ((uint32_t)(kRRows >> 4) << 24);
     static constexpr uint32_t IDESC_PV = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
@@ -88,7 +100,7 @@ struct RCfg {
 };
 
 struct RouteParams {
-    CUtensorMap tm_k, tm_v;             // [B*heads*N, D] bf16 natural order, box {64, 128}
+    CUtensorMap tm_k, tm_v;             // [B*heads*N, D] bf16 natural order, box {64, 64}
     const __nv_bfloat16* q;             // [B*heads*N, D]
     const int32_t* rows;                // [R] sampled natural tokens
     const vsa_mask_spec* cand;          // [2][heads]
@@ -100,55 +112,75 @@ struct RouteParams {
 };
 
 // Bits [lo, hi) of a 32-key word, lo and hi relative to the word start.
-__device__ __forceinline__ uint32_t span_bits(int lo, int hi)
+__device__ __forceinline__ uint32_t span32(int lo, int hi)
 {
     lo = max(lo, 0);
     hi = min(hi, 32);
-    if (hi <= lo) return 0u;
-    return (uint32_t)(((1ull << hi) - 1ull) ^ ((1ull << lo) - 1ull));
+    const int d = hi - lo;                        // 0 < d <= 32 and 0 <= lo < 32 when kept
+    return d > 0 ? (0xFFFFFFFFu >> (32 - d)) << lo : 0u;
 }
 
-// OR the natural-key interval [lo, hi) into the tile's keep words (tile keys
-// start at k0).
-__device__ __forceinline__ void or_span(uint32_t (&w)[kRBK / 32], long long k0, long long lo, long long hi)
-{
-    const long long a = lo - k0, b = hi - k0;
-    if (b <= 0 || a >= kRBK) return;
-#pragma unroll
-    for (int i = 0; i < kRBK / 32; ++i) w[i] |= span_bits((int)max(a - 32 * i, -1LL), (int)min(b - 32 * i, 33LL));
-}
+// Keep words of one sampled row over a walk of 32-key words (natural keys
+// [kw, kw + 32), kw advancing by a fixed stride), for the spatial candidate
+// (|t_k - tq| <= rt) and the temporal candidate (|h_k - hq| <= rh and
+// |w_k - wq| <= rw), each also keeping frame 0 when its sink bit is set; keys
+// past N are dropped.  The latent row g = kw / W, the column c = kw mod W and
+// h = g mod H of the word start are carried from word to word, so a word
+// costs a few 32-bit operations per latent row it meets.
+struct RowWalk {
+    int kw, c, hr;                      // word start, its column, its h
+    int sp_lo, sp_hi, sink_hi_s, sink_hi_t;
+    int hq, rh, wlo, whi1;
+    int W, H, N;
 
-// Keep words of a sampled row (frame tq, row hq, column wq) over natural keys
-// [k0, k0 + 128) for the spatial candidate (|t_k - tq| <= rt) and the
-// temporal candidate (|h_k - hq| <= rh and |w_k - wq| <= rw), each also
-// keeping frame 0 when its sink bit is set.  Keys past N are dropped.
-__device__ __forceinline__ void route_row_bits(const vsa_mask_spec& ms, const vsa_mask_spec& mt, int T, int H,
-                                               int W, long long N, int tq, int hq, int wq, long long k0,
-                                               uint32_t (&sp)[kRBK / 32], uint32_t (&tm)[kRBK / 32])
-{
-    const long long HW = (long long)H * W;
-#pragma unroll
-    for (int i = 0; i < kRBK / 32; ++i) sp[i] = tm[i] = 0u;
-    if (ms.sink) or_span(sp, k0, 0, HW);
-    or_span(sp, k0, (long long)max(0, tq - ms.rt) * HW, (long long)min(T, tq + ms.rt + 1) * HW);
-    if (mt.sink) or_span(tm, k0, 0, HW);
-    // latent rows g = t*H + h that meet the tile: keep columns |w - wq| <= rw
-    const long long wlo = max(0, wq - mt.rw), whi = min(W - 1, wq + mt.rw) + 1;
-    const long long g1 = min(k0 + kRBK, N) - 1;
-    for (long long g = k0 / W; g * W <= g1; ++g) {
-        const int h = (int)(g % H);
-        if (h - hq <= mt.rh && hq - h <= mt.rh) or_span(tm, k0, g * W + wlo, g * W + whi);
+    __device__ __forceinline__ void init(const vsa_mask_spec& ms, const vsa_mask_spec& mt, int T, int Hh, int Wd,
+                                         int Nn, int tq, int hq_, int wq, int kw0)
+    {
+        const int HW = Hh * Wd;
+        W = Wd;
+        H = Hh;
+        N = Nn;
+        kw = kw0;
+        c = kw0 % Wd;
+        hr = (kw0 / Wd) % Hh;
+        sp_lo = max(0, tq - ms.rt) * HW;
+        sp_hi = min(T, tq + min(ms.rt, T) + 1) * HW;
+        sink_hi_s = ms.sink ? HW : 0;
+        sink_hi_t = mt.sink ? HW : 0;
+        hq = hq_;
+        rh = mt.rh;
+        wlo = max(0, wq - mt.rw);
+        whi1 = min(Wd - 1, wq + min(mt.rw, Wd)) + 1;
     }
-    if (k0 + kRBK > N) {
-        const int nreal = (int)(N - k0);
-#pragma unroll
-        for (int i = 0; i < kRBK / 32; ++i) {
-            const uint32_t r = span_bits(0, nreal - 32 * i);
-            sp[i] &= r;
-            tm[i] &= r;
+
+    __device__ __forceinline__ void bits(uint32_t& sp, uint32_t& tm) const
+    {
+        sp = kw < sink_hi_s ? span32(-kw, sink_hi_s - kw) : 0u;
+        if (kw < sp_hi && kw + 32 > sp_lo) sp |= span32(sp_lo - kw, sp_hi - kw);
+        tm = kw < sink_hi_t ? span32(-kw, sink_hi_t - kw) : 0u;
+        int hh = hr;
+        for (int off = -c; off < 32; off += W) {
+            const int dh = hh - hq;
+            if (dh <= rh && -dh <= rh) tm |= span32(off + wlo, off + whi1);
+            if (++hh == H) hh = 0;
+        }
+        if (kw + 32 > N) {
+            const uint32_t real = span32(0, N - kw);
+            sp &= real;
+            tm &= real;
         }
     }
-}
+
+    __device__ __forceinline__ void advance(int stride)
+    {
+        kw += stride;
+        c += stride;
+        while (c >= W) {
+            c -= W;
+            if (++hr == H) hr = 0;
+        }
+    }
+};
 
 template <int D>
 __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __grid_constant__ RouteParams P)
@@ -176,10 +208,12 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
     auto BAR_VF = [&](int s) { return bar0 + 8u * (2 * C::STAGES + s); };
     auto BAR_VE = [&](int s) { return bar0 + 8u * (3 * C::STAGES + s); };
     const uint32_t BAR_QF = bar0 + 8u * (4 * C::STAGES);
-    const uint32_t BAR_SF = BAR_QF + 8u;
-    const uint32_t BAR_PF = BAR_QF + 16u;
-    const uint32_t BAR_PV = BAR_QF + 24u;
-    const uint32_t BAR_DR = BAR_QF + 32u;
+    auto BAR_SF = [&](int x) { return BAR_QF + 8u * (1 + x); };
+    auto BAR_PF = [&](int x) { return BAR_QF + 8u * (3 + x); };
+    const uint32_t BAR_PV = BAR_QF + 40u;
+    const uint32_t BAR_DR = BAR_QF + 48u;
+    const uint32_t BAR_FIN = BAR_QF + 56u;        // one phase: every MMA of the CTA complete
+    auto BAR_SC = [&](int x) { return BAR_QF + 8u * (8 + x); };   // all 8 softmax warps read S_x
     uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
     volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
     volatile int* issued = (volatile int*)(smem + C::OFF_MISC + 8);   // K copies, V copies, MMAs
@@ -193,10 +227,14 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
             mbar_init(BAR_VE(s), 1);
         }
         mbar_init(BAR_QF, 128);                 // the four gathering warps' threads
-        mbar_init(BAR_SF, 1);
-        mbar_init(BAR_PF, 4);                   // the four softmax warps
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR_SF(x), 1);
+            mbar_init(BAR_PF(x), kRSoftmaxWarps);
+        }
         mbar_init(BAR_PV, 1);
         mbar_init(BAR_DR, 1);
+        mbar_init(BAR_FIN, 1);
+        for (int x = 0; x < 2; ++x) mbar_init(BAR_SC(x), kRSoftmaxWarps);
         *abort_flag = 0;
         issued[0] = issued[1] = issued[2] = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -214,11 +252,11 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp >= 4) {
+    if (warp >= kRProducerWarp) {
         // ---- gather the sampled q rows: thread i -> row i, 16-byte chunks
         // into the 128-byte-swizzled K-major layout (chunk u of row i at
         // u ^ (i mod 8)), in D/64 column blocks of 128 rows x 128 bytes
-        const int i = threadIdx.x - 128;
+        const int i = threadIdx.x - 32 * kRProducerWarp;
         int tok = __ldg(P.rows + min(rt * kRRows + i, P.R - 1));
         if (tok < 0 || tok >= P.N) {
             atomicOr(P.status, VSA_DEV_BADSTATE);
@@ -265,7 +303,7 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
         if (mbar_wait_warp(BAR_QF, 0, ctl)) {
             tc_fence_after();
             const uint64_t qdesc = smem_desc(s_base + C::OFF_Q, 16, 1024);
-            const uint64_t pdesc = smem_desc(s_base + C::OFF_P, 16, 1024);
+            const uint64_t pdesc0 = smem_desc(s_base + C::OFF_P, 16, 1024);
             const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
             const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, kRBK * 128, 1024);
             constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
@@ -277,102 +315,122 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
                 const int st = j % C::STAGES;
                 if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES) & 1, ctl)) return false;
                 tc_fence_after();
+                const uint32_t dS = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
                 const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
-                mma_ss_lead<0>(tmem + C::COL_S, qdesc, kd, C::IDESC_QK, leader);
+                mma_ss_lead<0>(dS, qdesc, kd, C::IDESC_QK, leader);
 #pragma unroll
                 for (int kk = 1; kk < D / 16; ++kk)
-                    mma_ss_lead<1>(tmem + C::COL_S, qdesc + kstep(kk, kRRows), kd + kstep(kk, kRBK), C::IDESC_QK,
-                                   leader);
-                tc_commit_lead(BAR_SF, leader);
+                    mma_ss_lead<1>(dS, qdesc + kstep(kk, kRRows), kd + kstep(kk, kRBK), C::IDESC_QK, leader);
+                tc_commit_lead(BAR_SF(j & 1), leader);
                 tc_commit_lead(BAR_KE(st), leader);
                 return true;
             };
             bool go = issue_qk(0);
             if (go && leader) issued[2] = 1;
+            go = go && (n < 2 || issue_qk(1));
             for (int j = 0; go && j < n; ++j) {
-                const int vs = j % C::STAGES;
-                if (!mbar_wait_warp(BAR_PF, (uint32_t)j & 1, ctl)) break;
-                if (!mbar_wait_warp(BAR_VF(vs), (uint32_t)(j / C::STAGES) & 1, ctl)) break;
+                const int x = j & 1, vs = j % C::STAGES;
+                go = mbar_wait_warp(BAR_PF(x), (uint32_t)(j >> 1) & 1, ctl) &&
+                     mbar_wait_warp(BAR_VF(vs), (uint32_t)(j / C::STAGES) & 1, ctl);
+                if (!go) break;
                 tc_fence_after();
                 const uint64_t vd = vdesc0 + (uint64_t)vs * kStageStep;
-                // O_full += P_full V (P_full: TMEM columns [0, 64) of S)
-                if (j == 0) mma_ts_lead<0>(tmem + C::COL_OF, tmem + C::COL_S, vd, C::IDESC_PV, leader);
-                else mma_ts_lead<1>(tmem + C::COL_OF, tmem + C::COL_S, vd, C::IDESC_PV, leader);
+                const uint32_t aS = tmem + (x ? C::COL_S1 : C::COL_S0);
+                const uint64_t pd = pdesc0 + (uint64_t)x * (C::P_BYTES >> 4);
+                // O_full += P_full V (TMEM columns [0, 32) of S_x), O_sp += P_sp V
+                // ([32, 64)), O_tm += P_tm V (shared memory); the first tile of
+                // the CTA initialises the accumulators
 #pragma unroll
-                for (int kk = 1; kk < kRBK / 16; ++kk)
-                    mma_ts_lead<1>(tmem + C::COL_OF, tmem + C::COL_S + kk * 8,
-                                   vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
-                // O_sp += P_sp V (P_sp: TMEM columns [64, 128))
-                if (j == 0) mma_ts_lead<0>(tmem + C::COL_OS, tmem + C::COL_S + 64, vd, C::IDESC_PV, leader);
-                else mma_ts_lead<1>(tmem + C::COL_OS, tmem + C::COL_S + 64, vd, C::IDESC_PV, leader);
-#pragma unroll
-                for (int kk = 1; kk < kRBK / 16; ++kk)
-                    mma_ts_lead<1>(tmem + C::COL_OS, tmem + C::COL_S + 64 + kk * 8,
-                                   vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
-                // O_tm += P_tm V (P_tm in shared memory, K-major, swizzled)
-                if (j == 0) mma_ss_lead<0>(tmem + C::COL_OT, pdesc, vd, C::IDESC_PV, leader);
-                else mma_ss_lead<1>(tmem + C::COL_OT, pdesc, vd, C::IDESC_PV, leader);
-#pragma unroll
-                for (int kk = 1; kk < kRBK / 16; ++kk)
-                    mma_ss_lead<1>(tmem + C::COL_OT, pdesc + kstep(kk, kRRows),
-                                   vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
+                for (int kk = 0; kk < kRBK / 16; ++kk) {
+                    const uint64_t vk = vd + (uint64_t)((kk * 16 * 128) >> 4);
+                    if (j == 0 && kk == 0) {
+                        mma_ts_lead<0>(tmem + C::COL_OF, aS, vk, C::IDESC_PV, leader);
+                        mma_ts_lead<0>(tmem + C::COL_OF + D, aS + 32, vk, C::IDESC_PV, leader);
+                        mma_ss_lead<0>(tmem + C::COL_OF + 2 * D, pd, vk, C::IDESC_PV, leader);
+                    } else {
+                        mma_ts_lead<1>(tmem + C::COL_OF, aS + kk * 8, vk, C::IDESC_PV, leader);
+                        mma_ts_lead<1>(tmem + C::COL_OF + D, aS + 32 + kk * 8, vk, C::IDESC_PV, leader);
+                        mma_ss_lead<1>(tmem + C::COL_OF + 2 * D, pd + (uint64_t)(kk * 2), vk, C::IDESC_PV, leader);
+                    }
+                }
                 tc_commit_lead(BAR_PV, leader);
                 tc_commit_lead(BAR_VE(vs), leader);
-                // the next S overwrites P_full / P_sp: queued behind the PV MMAs
-                if (j + 1 < n) go = issue_qk(j + 1);
+                // S_{j+2} reuses S_x: queued behind PV_j, so P_j is read first
+                if (j + 2 < n) go = issue_qk(j + 2);
             }
+            // a single-phase barrier for the epilogue (the PV barrier's parity
+            // cannot tell its last phase from the one before)
+            if (go) tc_commit_lead(BAR_FIN, leader);
         }
-    } else if (warp < 4) {
-        // ---------------- softmax: thread r owns sampled row r ----------------
-        const int r = threadIdx.x;
-        const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
-        const uint32_t tS = tmem + lane_off + C::COL_S;
+    } else if (warp < kRSoftmaxWarps) {
+        // ---------------- softmax: warpgroup G, thread r owns sampled row r ----------------
+        const int G = warp >> 2;
+        const int r = threadIdx.x & (kRRows - 1);
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
         int tok = __ldg(P.rows + min(rt * kRRows + r, P.R - 1));
         if (tok < 0 || tok >= P.N) tok = 0;              // flagged by the gather
         const int HW = P.H * P.W;
         const int tq = tok / HW, hq = (tok % HW) / P.W, wq = tok % P.W;
-        const vsa_mask_spec ms = P.cand[head];
-        const vsa_mask_spec mt = P.cand[P.heads + head];
+        RowWalk walk;
+        walk.init(P.cand[head], P.cand[P.heads + head], P.T, P.H, P.W, P.N, tq, hq, wq, j0 * kRBK + 32 * G);
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
-        float m_run = -INFINITY;                          // log2 units, shared by the three softmaxes
-        float lf = 0.0f, ls = 0.0f, lt = 0.0f;
+        float* sums = (float*)(smem + C::OFF_SUM);        // [G][3][row]
+        float m_run = -INFINITY;                          // log2 units, identical in both warpgroups
+        float lf = 0.0f, ls = 0.0f, lt = 0.0f;            // this warpgroup's keys only
         bool ok = true;
-        for (int j = 0; j < n; ++j) {
-            const long long k0 = (long long)(j0 + j) * kRBK;
-            uint32_t bsp[kRBK / 32], btm[kRBK / 32];
-            route_row_bits(ms, mt, P.T, P.H, P.W, P.N, tq, hq, wq, k0, bsp, btm);
-            if (!mbar_wait_warp(BAR_SF, (uint32_t)j & 1, ctl)) { ok = false; break; }
+        for (int j = 0; j < n && ok; ++j) {
+            const int x = j & 1;
+            const uint32_t tS = tmem + lane_off + (x ? C::COL_S1 : C::COL_S0);
+            const int left = P.N - (walk.kw - 32 * G);    // real keys of the tile (>= 1)
+            uint32_t ws, wt;
+            walk.bits(ws, wt);
+            walk.advance(kRBK);
+            if (!mbar_wait_warp(BAR_SF(x), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
-            float s[kRBK];
+            // both warpgroups read the whole tile: the row max needs all 64
+            // keys, and each exponentiates its own 32
+            float s[32];
+            float mx;
             {
-                uint32_t sr[kRBK];
-#pragma unroll
-                for (int c = 0; c < kRBK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+                uint32_t sr[32], so[32];
+                tmem_ld32(tS + 32 * G, sr);
+                tmem_ld32(tS + 32 * (G ^ 1), so);
                 tmem_ld_wait();
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(BAR_SC(x));    // S_x read: P may overwrite it
 #pragma unroll
-                for (int c = 0; c < kRBK; ++c) {
+                for (int c = 0; c < 32; ++c) {
                     reg_fence(sr[c]);
+                    reg_fence(so[c]);
                     s[c] = __uint_as_float(sr[c]);
                 }
+                float b;
+                if (left >= kRBK) {                       // every key real (all but the last tile)
+                    float a = s[0], a2 = __uint_as_float(so[0]);
+#pragma unroll
+                    for (int c = 1; c < 31; c += 2) {
+                        a = max3(a, s[c], s[c + 1]);
+                        a2 = max3(a2, __uint_as_float(so[c]), __uint_as_float(so[c + 1]));
+                    }
+                    a = max3(a, s[31], a2);
+                    b = __uint_as_float(so[31]);
+                    mx = fmaxf(a, b);
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (32 * G + c >= left) s[c] = -INFINITY;
+                    float a = s[0];
+#pragma unroll
+                    for (int c = 1; c < 32; ++c) a = fmaxf(a, s[c]);
+                    b = -INFINITY;
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (32 * (G ^ 1) + c < left) b = fmaxf(b, __uint_as_float(so[c]));
+                    mx = fmaxf(a, b);
+                }
             }
-            const long long left = (long long)P.N - k0;
-            if (left < kRBK) {
-#pragma unroll
-                for (int c = 0; c < kRBK; ++c)
-                    if (c >= left) s[c] = -INFINITY;
-            }
-            float mc[kRBK / 32];
-#pragma unroll
-            for (int g = 0; g < kRBK / 32; ++g) {
-                float a = s[g * 32];
-#pragma unroll
-                for (int c = 1; c < 31; c += 2) a = max3(a, s[g * 32 + c], s[g * 32 + c + 1]);
-                mc[g] = fmaxf(a, s[g * 32 + 31]);
-            }
-            float mx = mc[0];
-#pragma unroll
-            for (int g = 1; g < kRBK / 32; ++g) mx = fmaxf(mx, mc[g]);
             const float mxs = mx * sl;                    // finite: every tile holds a real key
             float alpha = 1.0f;
             bool need_o = false;
@@ -386,11 +444,14 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
                 m_run = mxs;
                 need_o = true;
             }
-            // S_j complete implies the PV MMAs of tile j-1 are complete (one
-            // thread issues them in order), so O and P_tm may be touched now
             if (__any_sync(0xFFFFFFFFu, need_o)) {
+                // the accumulators still take PV_{j-1}: wait for it, then this
+                // warpgroup rescales its half of the 3 D columns
+                ok = mbar_wait_warp(BAR_PV, (uint32_t)(j - 1) & 1, ctl);
+                if (!ok) break;
+                tc_fence_after();
 #pragma unroll 1
-                for (int c = 0; c < 3 * D / 32; ++c) {
+                for (int c = G * (3 * D / 64); c < (G + 1) * (3 * D / 64); ++c) {
                     uint32_t ov[32];
                     const uint32_t ta = tmem + lane_off + C::COL_OF + c * 32;
                     tmem_ld32(ta, ov);
@@ -405,61 +466,102 @@ __global__ void __launch_bounds__(kRThreads, 1) route_partial_kernel(const __gri
             }
             const float mneg = -m_run;
             const unsigned long long mneg2 = f2_pack(mneg, mneg);
+            float p[32];
+            uint32_t pf[16], ps[16], pt[16];
+            unsigned long long af2 = 0ull;                // packed pair sums
 #pragma unroll
-            for (int cc = 0; cc < kRBK / 32; ++cc) {
-                uint32_t pf[16], ps[16], pt[16];
-                const uint32_t ws = bsp[cc], wt = btm[cc];
-                float af = 0.0f, as = 0.0f, at = 0.0f;
+            for (int i = 0; i < 16; ++i) {
+                float x0, x1;
+                f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2, mneg2), x0, x1);
+                p[2 * i] = ex2(x0);
+                p[2 * i + 1] = ex2(x1);
+                af2 = f2_add(af2, f2_pack(p[2 * i], p[2 * i + 1]));
+                pf[i] = pack_bf16(p[2 * i], p[2 * i + 1]);
+            }
+            float af, af1;
+            f2_unpack(af2, af, af1);
+            af += af1;
+            lf += af;
+            // spatial keep bits are usually all set or all clear across the
+            // warp (the sampled rows are sorted, so a warp's rows share frames)
+            if (__all_sync(0xFFFFFFFFu, ws == 0xFFFFFFFFu)) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ps[i] = pf[i];
+                ls += af;
+            } else if (__all_sync(0xFFFFFFFFu, ws == 0u)) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) ps[i] = 0u;
+            } else {
+                unsigned long long a2 = 0ull;
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(s[cc * 32 + 2 * i], s[cc * 32 + 2 * i + 1]), sl2, mneg2), x0, x1);
-                    const float p0 = ex2(x0), p1 = ex2(x1);
-                    const float s0 = ((ws >> (2 * i)) & 1u) ? p0 : 0.0f;
-                    const float s1 = ((ws >> (2 * i + 1)) & 1u) ? p1 : 0.0f;
-                    const float t0 = ((wt >> (2 * i)) & 1u) ? p0 : 0.0f;
-                    const float t1 = ((wt >> (2 * i + 1)) & 1u) ? p1 : 0.0f;
-                    af += p0 + p1;
-                    as += s0 + s1;
-                    at += t0 + t1;
-                    pf[i] = pack_bf16(p0, p1);
+                    const float s0 = (ws & (1u << (2 * i))) ? p[2 * i] : 0.0f;
+                    const float s1 = (ws & (1u << (2 * i + 1))) ? p[2 * i + 1] : 0.0f;
+                    a2 = f2_add(a2, f2_pack(s0, s1));
                     ps[i] = pack_bf16(s0, s1);
+                }
+                float a0, a1;
+                f2_unpack(a2, a0, a1);
+                ls += a0 + a1;
+            }
+            if (__all_sync(0xFFFFFFFFu, wt == 0u)) {
+#pragma unroll
+                for (int i = 0; i < 16; ++i) pt[i] = 0u;
+            } else {
+                unsigned long long a2 = 0ull;
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float t0 = (wt & (1u << (2 * i))) ? p[2 * i] : 0.0f;
+                    const float t1 = (wt & (1u << (2 * i + 1))) ? p[2 * i + 1] : 0.0f;
+                    a2 = f2_add(a2, f2_pack(t0, t1));
                     pt[i] = pack_bf16(t0, t1);
                 }
-                lf += af;
-                ls += as;
-                lt += at;
-                tmem_st16(tS + cc * 16, pf);              // P_full: S columns [0, 64)
-                tmem_st16(tS + 64 + cc * 16, ps);         // P_sp:   S columns [64, 128)
-                // P_tm keys [32cc, 32cc + 32): block cc/2, chunks 4(cc%2)..+3 of row r
+                float a0, a1;
+                f2_unpack(a2, a0, a1);
+                lt += a0 + a1;
+            }
+            // S_j complete implies PV_{j-2} complete, the last reader of S_x's
+            // P columns and of P_tm buffer x; the other warpgroup must have
+            // read its S_x columns too
+            ok = mbar_wait_warp(BAR_SC(x), (uint32_t)(j >> 1) & 1, ctl);
+            if (!ok) break;
+            tc_fence_after();
+            tmem_st16(tS + 16 * G, pf);                   // P_full: S_x columns [0, 32)
+            tmem_st16(tS + 32 + 16 * G, ps);              // P_sp:   S_x columns [32, 64)
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int chunk = (cc & 1) * 4 + u;
-                    const uint32_t dst = s_base + C::OFF_P + (cc >> 1) * (kRRows * 128) + r * 128 +
-                                         ((chunk ^ (r & 7)) << 4);
-                    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pt[4 * u]),
-                                 "r"(pt[4 * u + 1]), "r"(pt[4 * u + 2]), "r"(pt[4 * u + 3])
-                                 : "memory");
-                }
+            for (int u = 0; u < 4; ++u) {
+                const int chunk = 4 * G + u;              // keys 32G + 8u .. + 8 of row r
+                const uint32_t dst = s_base + C::OFF_P + x * C::P_BYTES + r * 128 + ((chunk ^ (r & 7)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pt[4 * u]),
+                             "r"(pt[4 * u + 1]), "r"(pt[4 * u + 2]), "r"(pt[4 * u + 3])
+                             : "memory");
             }
             tmem_st_wait();
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(BAR_PF);
+            if (lane == 0) mbar_arrive(BAR_PF(x));
         }
 
         // ---------------- partial record of this CTA ----------------
-        bool have = ok && mbar_wait_warp(BAR_PV, (uint32_t)(n - 1) & 1, ctl);
+        const bool have = ok && mbar_wait_warp(BAR_FIN, 0, ctl);
         tc_fence_after();
+        sums[(G * 3 + 0) * kRRows + r] = lf;
+        sums[(G * 3 + 1) * kRRows + r] = ls;
+        sums[(G * 3 + 2) * kRRows + r] = lt;
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kRSoftmaxWarps) : "memory");
         float* rec = P.part + ((size_t)unit * P.S + split) * C::PART_FLOATS;
-        rec[r] = have ? m_run : -INFINITY;
-        rec[kRRows + r] = have ? lf : 0.0f;
-        rec[2 * kRRows + r] = have ? ls : 0.0f;
-        rec[3 * kRRows + r] = have ? lt : 0.0f;
+        const bool all = !*abort_flag && have;
+        if (G == 0) {
+            rec[r] = all ? m_run : -INFINITY;
+#pragma unroll
+            for (int k = 0; k < 3; ++k)
+                rec[(1 + k) * kRRows + r] = all ? sums[k * kRRows + r] + sums[(3 + k) * kRRows + r] : 0.0f;
+        }
         if (have) {
+            // warpgroup G writes its half of the 3 D accumulator columns
 #pragma unroll 1
-            for (int c = 0; c < 3 * D / 32; ++c) {
+            for (int c = G * (3 * D / 64); c < (G + 1) * (3 * D / 64); ++c) {
                 uint32_t ov[32];
                 tmem_ld32(tmem + lane_off + C::COL_OF + c * 32, ov);
                 tmem_ld_wait();
@@ -608,7 +710,7 @@ struct RouteShape {
     size_t part_bytes, err_bytes;
 };
 
-// Splits of the key range: fewest waves x tiles per CTA (+4 tiles of fixed
+// Splits of the key range: fewest waves x tiles per CTA (+8 tiles of fixed
 // cost for the gather and the ~200 KB partial record), the smaller split on a
 // tie.
 int choose_splits(long long units, int nK, int sms)
@@ -618,7 +720,7 @@ int choose_splits(long long units, int nK, int sms)
     const int smax = nK < kRMaxSplits ? nK : kRMaxSplits;
     for (int s = 1; s <= smax; ++s) {
         const long long waves = (units * s + sms - 1) / sms;
-        const long long cost = waves * ((nK + s - 1) / s + 4);
+        const long long cost = waves * ((nK + s - 1) / s + 8);
         if (best_cost < 0 || cost < best_cost) {
             best_cost = cost;
             best = s;
@@ -632,7 +734,7 @@ int route_shape(vsa_plan_t plan, int B, int D, int n_rows, RouteShape* out)
     if (!plan || B < 1 || n_rows < 1) return VSA_ERR_INVALID_ARG;
     if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
     const vsa_dims& d = plan->d;
-    if ((long long)B * d.heads * d.N > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
+    if ((long long)B * d.heads * d.N + 2 * kRBK > 0x7FFFFFFFLL) return VSA_ERR_UNSUPPORTED;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
