@@ -85,6 +85,8 @@ def _load() -> ctypes.CDLL:
         "vsa_svg_route_workspace_size": ([vp, i32, i32, i32, P(sz)], i32),
         "vsa_svg_route": ([vp, vp, vp, vp, i32, i32, vp, i32, f32, vp, vp, vp, sz, vp], i32),
         "vsa_plan_apply_route": ([vp, vp, vp], i32),
+        "vsa_ulysses_permute": ([vp, vp, i32, i32, i32, i32, vp, P(vp), vp], i32),
+        "vsa_ulysses_unpermute": ([vp, vp, i32, i32, i32, i32, vp, P(vp), vp], i32),
         "vsa_status_string": ([i32], ctypes.c_char_p),
         "vsa_version": ([], i32),
     }
@@ -283,6 +285,27 @@ def vsa_svg_route(plan: int, q, k, v, B: int, D: int, rows, n_rows: int, scale: 
     _check(_lib.vsa_svg_route(plan, _ptr(q), _ptr(k), _ptr(v), B, D, _ptr(rows), n_rows, scale,
                               _ptr(err), _ptr(flags), _ptr(workspace), workspace_bytes,
                               _stream(stream)), "vsa_svg_route")
+
+
+def _ptr_array(ptrs) -> "ctypes.Array":
+    return (ctypes.c_void_p * len(ptrs))(*[_ptr(p) for p in ptrs])
+
+
+def vsa_ulysses_permute(plan: int, x, B: int, D: int, rank: int, world: int, head_layout, dst,
+                        stream=None) -> None:
+    _check(_lib.vsa_ulysses_permute(plan, _ptr(x), B, D, rank, world, _ptr(head_layout), _ptr_array(dst),
+                                    _stream(stream)), "vsa_ulysses_permute")
+
+
+def vsa_ulysses_unpermute(plan: int, o, B: int, D: int, rank: int, world: int, head_layout, dst,
+                          stream=None) -> None:
+    _check(_lib.vsa_ulysses_unpermute(plan, _ptr(o), B, D, rank, world, _ptr(head_layout), _ptr_array(dst),
+                                      _stream(stream)), "vsa_ulysses_unpermute")
+
+
+def shard_offsets(n_tokens: int, world: int) -> list:
+    """Token offsets of the sequence shards: rank r holds [off[r], off[r+1])."""
+    return [r * n_tokens // world for r in range(world + 1)]
 
 
 def vsa_plan_apply_route(plan: int, flags, stream=None) -> None:

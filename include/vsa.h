@@ -13,6 +13,8 @@
  *   vsa_unpermute     o  tile-major -> natural [B,Hh,N,D]
  *   vsa_svg_route     sampled-query profiling -> per-head spatial / temporal
  *                     flags; vsa_plan_apply_route switches the heads' specs
+ *   vsa_ulysses_permute / _unpermute  sequence-sharded <-> head-sharded
+ *                     exchange fused with the token order, across GPUs
  *
  * Sources (web pages on block-sparse video attention):
  *  [SVG-TPU] "Sparse VideoGen: accelerating video diffusion attention on TPU"
@@ -298,6 +300,40 @@ int vsa_svg_route(vsa_plan_t plan, const void* q, const void* k, const void* v,
  * (n_slots, list capacity) are unchanged; vsa_permute / vsa_unpermute pick
  * each head's token order from the new specs.  Asynchronous, capturable. */
 int vsa_plan_apply_route(vsa_plan_t plan, const int32_t* flags, void* stream);
+
+/* ---- Head-sharded attention across GPUs ---------------------------------
+ * [SVG-TPU] "performing layout transformation on local heads": inputs
+ * arrive sequence-sharded, an all-to-all gives every rank all tokens of its
+ * heads ([B,S/N,H,D] -> [B,S,H/N,D]), each rank permutes its heads' tokens
+ * after that exchange, runs attention, restores the order and exchanges
+ * back.  Here exchange and permutation are one pass each way, through the
+ * other ranks' memory (peer stores over NVLink).
+ *
+ * world ranks (1..8), rank r holds the natural tokens [off_r, off_{r+1}),
+ * off_r = floor(r * N / world), of all world*num_heads heads; rank g owns
+ * global heads [g*num_heads, (g+1)*num_heads) and `plan` is its plan (its
+ * heads' specs, the full grid).  head_layout: device int32 [world*num_heads],
+ * the token order (vsa_layout) of every global head, equal to each owner's
+ * plan spec.  dst: host array of `world` device pointers (16-byte aligned),
+ * entry g addressable from this GPU (rank g's buffer, or a local one when
+ * every rank lives on this GPU).
+ *
+ * vsa_ulysses_permute: x = this rank's shard bf16 [B][n_rank][world*heads][D]
+ * -> dst[g] = rank g's tile-major q/k/v [B][num_heads][n_slots][D]: every
+ * (token, head) row goes to its owner at the token's slot; this rank also
+ * zeroes the padding slots of its own buffer dst[rank].
+ * vsa_ulysses_unpermute: o = this rank's tile-major output
+ * [B][num_heads][n_slots][D] -> dst[r] = rank r's output shard
+ * [B][n_r][world*heads][D], each token to its owner.
+ *
+ * The kernels wait on no other rank.  The caller orders them: every rank's
+ * exchange must be complete before any rank reads the buffers it wrote (a
+ * collective on the stream after each exchange), and a rank's buffers must
+ * not be rewritten while it still reads them.  Asynchronous. */
+int vsa_ulysses_permute(vsa_plan_t plan, const void* x, int B, int D, int rank, int world,
+                        const int32_t* head_layout, void* const* dst, void* stream);
+int vsa_ulysses_unpermute(vsa_plan_t plan, const void* o, int B, int D, int rank, int world,
+                          const int32_t* head_layout, void* const* dst, void* stream);
 
 /* Synchronises `stream`, then reports and clears the plan's device status
  * word: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_DEVICE; VSA_ERR_CUDA if the

@@ -282,3 +282,38 @@ def svg_route(spatial_specs, temporal_specs, grid, D: int, scale: float,
     err /= float(B * len(rows) * D)
     flags = (err[:, 1] < err[:, 0]).astype(np.int32)
     return err, flags
+
+
+def shard_offsets(n_tokens: int, world: int):
+    """Sequence shards of the head-sharded exchange: rank r holds natural
+    tokens [off[r], off[r+1]), off[r] = floor(r * N / world)."""
+    return [r * n_tokens // world for r in range(world + 1)]
+
+
+def ulysses_exchange(x: np.ndarray, world: int):
+    """The all-to-all of head-sharded attention ("Sparse VideoGen:
+    accelerating video diffusion attention on TPU", "performing layout
+    transformation on local heads": [B,S/N,H,D] -> [B,S,H/N,D]), written out
+    from its definition.  x: [B, Hh, N, D] (natural token order).  Returns
+    (shards, head_local): shards[r] = [B, n_r, Hh, D], the tokens rank r
+    holds for every head; head_local[g] = [B, Hh/world, N, D], every token of
+    rank g's heads [g Hh/world, (g+1) Hh/world)."""
+    B, Hh, N, D = x.shape
+    assert Hh % world == 0
+    off = shard_offsets(N, world)
+    hpr = Hh // world
+    shards = [np.ascontiguousarray(x[:, :, off[r]:off[r + 1], :].transpose(0, 2, 1, 3)) for r in range(world)]
+    head_local = [np.ascontiguousarray(x[:, g * hpr:(g + 1) * hpr]) for g in range(world)]
+    return shards, head_local
+
+
+def layout_gather(x_head_local: np.ndarray, perms) -> np.ndarray:
+    """[B, heads, N, D] natural order -> [B, heads, n_slots, D] in each head's
+    slot order (perms[h][p] = natural token of slot p, -1 = padding -> 0)."""
+    B, Hh, N, D = x_head_local.shape
+    S = len(perms[0])
+    out = np.zeros((B, Hh, S, D), dtype=x_head_local.dtype)
+    for h in range(Hh):
+        real = perms[h] >= 0
+        out[:, h, real] = x_head_local[:, h, perms[h][real]]
+    return out

@@ -96,6 +96,8 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_svg_route_workspace_size(None, 1, 128, 1, ctypes.byref(n)) == -1
     assert L.vsa_svg_route(None, None, None, None, 1, 128, None, 1, 0.1, None, None, None, 0, None) == -1
     assert L.vsa_plan_apply_route(None, None, None) == -1
+    assert L.vsa_ulysses_permute(None, None, 1, 128, 0, 1, None, None, None) == -1
+    assert L.vsa_ulysses_unpermute(None, None, 1, 128, 0, 1, None, None, None) == -1
 
 
 def test_layout_slot_counts():
