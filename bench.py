@@ -294,7 +294,7 @@ def run_gpu(args, w, world, rank, local):
     sh = stream.cuda_stream
     has_stripe = any(s["kind"] == W.MASK_KINDS["stripe"] for s in w.specs)
     per_step_launches = (LAUNCHES["plan_build_stripe"] if has_stripe else LAUNCHES["plan_build"]) \
-        + 3 * LAUNCHES["permute"] + LAUNCHES["fwd"] + LAUNCHES["unpermute"]
+        + LAUNCHES["permute"] + LAUNCHES["fwd"] + LAUNCHES["unpermute"]
 
     # SVG routing before the plan build: sampled-query profiling, then the
     # per-head switch (which rebuilds the plan on the device)
@@ -331,9 +331,7 @@ def run_gpu(args, w, world, rank, local):
 
     def step(record_fwd: bool):
         plan_step(q, k, v, record_fwd)
-        vsa.vsa_permute(h, q, qp, B, w.D, sh)
-        vsa.vsa_permute(h, k, kp, B, w.D, sh)
-        vsa.vsa_permute(h, v, vp, B, w.D, sh)
+        vsa.vsa_permute_qkv(h, q, k, v, qp, kp, vp, B, w.D, sh)
         if record_fwd:
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
@@ -395,9 +393,7 @@ def run_gpu(args, w, world, rank, local):
         kd.copy_(pinned[1], non_blocking=True)
         vd.copy_(pinned[2], non_blocking=True)
         plan_step(qd, kd, vd, False)
-        vsa.vsa_permute(h, qd, qp, B, w.D, sh)
-        vsa.vsa_permute(h, kd, kp, B, w.D, sh)
-        vsa.vsa_permute(h, vd, vp, B, w.D, sh)
+        vsa.vsa_permute_qkv(h, qd, kd, vd, qp, kp, vp, B, w.D, sh)
         vsa.vsa_sparse_attn_fwd(qp, kp, vp, op, lse, h, B, w.D, w.scale, sh)
         vsa.vsa_unpermute(h, op, o, B, w.D, sh)
         o_host.copy_(o, non_blocking=True)

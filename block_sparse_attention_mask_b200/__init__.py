@@ -76,6 +76,7 @@ def _load() -> ctypes.CDLL:
         "vsa_plan_destroy": ([vp], i32),
         "vsa_permute": ([vp, vp, vp, i32, i32, vp], i32),
         "vsa_unpermute": ([vp, vp, vp, i32, i32, vp], i32),
+        "vsa_permute_qkv": ([vp, vp, vp, vp, vp, vp, vp, i32, i32, vp], i32),
         "vsa_sparse_attn_fwd": ([vp, vp, vp, vp, vp, vp, i32, i32, f32, vp], i32),
         "vsa_check_status": ([vp, vp], i32),
         "vsa_selftest_watchdog": ([vp, ctypes.c_longlong, vp], i32),
@@ -226,6 +227,11 @@ def vsa_permute(plan: int, x_in, x_out, B: int, D: int, stream=None) -> None:
 def vsa_unpermute(plan: int, x_in, x_out, B: int, D: int, stream=None) -> None:
     _check(_lib.vsa_unpermute(plan, _ptr(x_in), _ptr(x_out), int(B), int(D), _stream(stream)),
            "vsa_unpermute")
+
+
+def vsa_permute_qkv(plan: int, q, k, v, q_out, k_out, v_out, B: int, D: int, stream=None) -> None:
+    _check(_lib.vsa_permute_qkv(plan, _ptr(q), _ptr(k), _ptr(v), _ptr(q_out), _ptr(k_out), _ptr(v_out), B, D,
+                                _stream(stream)), "vsa_permute_qkv")
 
 
 def vsa_sparse_attn_fwd(q, k, v, o, lse, plan: int, B: int, D: int, scale: float,
@@ -418,11 +424,20 @@ def sparse_attn_fwd(plan: Plan, q, k, v, scale: Optional[float] = None, o=None, 
     return o, lse
 
 
+def permute_qkv(plan: Plan, q, k, v, stream=None):
+    """natural [B, Hh, N, D] x3 -> tile-major [B, Hh, n_slots, D] x3 in one launch."""
+    import torch
+    B, Hh, N, D = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        _require_bf16(t, (B, plan.heads, plan.n_tokens, D), name)
+    outs = [torch.empty((B, Hh, plan.n_slots, D), dtype=torch.bfloat16, device=q.device) for _ in range(3)]
+    vsa_permute_qkv(plan.handle, q, k, v, *outs, B, D, stream)
+    return tuple(outs)
+
+
 def attention(plan: Plan, q, k, v, scale: Optional[float] = None, stream=None):
     """Natural-order q, k, v [B, Hh, N, D] -> (o natural [B, Hh, N, D], lse tile-major)."""
-    qp = permute(plan, q, stream=stream)
-    kp = permute(plan, k, stream=stream)
-    vp = permute(plan, v, stream=stream)
+    qp, kp, vp = permute_qkv(plan, q, k, v, stream=stream)
     op, lse = sparse_attn_fwd(plan, qp, kp, vp, scale, stream=stream)
     return unpermute(plan, op, stream=stream), lse
 

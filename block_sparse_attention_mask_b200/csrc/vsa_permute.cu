@@ -63,6 +63,62 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_ma
     }
 }
 
+// q, k and v in one pass: the slot -> token arithmetic is done once per row
+// for the three tensors, and each thread keeps six 16-byte loads (two rows
+// of each tensor) in flight before its stores.
+template <int D>
+__global__ void __launch_bounds__(256) permute3_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                                       long long rows, const uint4* __restrict__ q,
+                                                       const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                       uint4* __restrict__ qo, uint4* __restrict__ ko,
+                                                       uint4* __restrict__ vo)
+{
+    constexpr int VPR = D * 2 / 16;
+    constexpr int RPW = 32 / VPR;
+    const int lane = threadIdx.x & 31;
+    const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+    const int sub = lane / VPR, c = lane % VPR;
+    const long long stride = nwarps * RPW;
+    for (long long r0 = warp * RPW + sub; r0 < rows; r0 += 2 * stride) {
+        long long src[2];
+        bool real[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const long long r = r0 + u * stride;
+            real[u] = false;
+            src[u] = 0;
+            if (r < rows) {
+                const long long bh = r / d.Nslots;
+                const long long p = r - bh * d.Nslots;
+                int t = 0, h = 0, w = 0;
+                const int layout = __ldg(&specs[bh % d.heads].layout);
+                if (vsa_slot_coords_any(d, layout, p, t, h, w)) {
+                    real[u] = true;
+                    src[u] = (bh * d.N + ((long long)t * d.H + h) * d.W + w) * VPR + c;
+                }
+            }
+        }
+        uint4 a[2], b[2], e[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+            a[u] = real[u] ? __ldg(q + src[u]) : z;
+            b[u] = real[u] ? __ldg(k + src[u]) : z;
+            e[u] = real[u] ? __ldg(v + src[u]) : z;
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const long long r = r0 + u * stride;
+            if (r < rows) {
+                qo[r * VPR + c] = a[u];
+                ko[r * VPR + c] = b[u];
+                vo[r * VPR + c] = e[u];
+            }
+        }
+    }
+}
+
 int sm_count()
 {
     static int cached = 0;
@@ -114,4 +170,45 @@ extern "C" int vsa_permute(vsa_plan_t plan, const void* in, void* out, int B, in
 extern "C" int vsa_unpermute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream)
 {
     return launch(false, plan, in, out, B, D, stream);
+}
+
+extern "C" int vsa_permute_qkv(vsa_plan_t plan, const void* q, const void* k, const void* v, void* q_out,
+                               void* k_out, void* v_out, int B, int D, void* stream)
+{
+    if (!plan || B < 0) return VSA_ERR_INVALID_ARG;
+    if (D != 64 && D != 128) return VSA_ERR_UNSUPPORTED;
+    if (B == 0) return VSA_OK;
+    const void* ins[3] = {q, k, v};
+    void* outs[3] = {q_out, k_out, v_out};
+    const vsa_dims& d = plan->d;
+    const long long rows = (long long)B * d.heads * d.Nslots;
+    const long long in_rows = (long long)B * d.heads * d.N;
+    const size_t row_bytes = (size_t)D * 2;
+    for (int i = 0; i < 3; ++i) {
+        if (!ins[i] || !outs[i]) return VSA_ERR_INVALID_ARG;
+        if (!vsa_aligned16(ins[i]) || !vsa_aligned16(outs[i])) return VSA_ERR_ALIGNMENT;
+    }
+    // no output may overlap an input or another output
+    for (int i = 0; i < 3; ++i)
+        for (int j = 0; j < 3; ++j) {
+            const char* ib = (const char*)ins[j];
+            const char* ob = (const char*)outs[i];
+            if (ib < ob + rows * row_bytes && ob < ib + in_rows * row_bytes) return VSA_ERR_INVALID_ARG;
+            if (i != j) {
+                const char* o2 = (const char*)outs[j];
+                if (o2 < ob + rows * row_bytes && ob < o2 + rows * row_bytes) return VSA_ERR_INVALID_ARG;
+            }
+        }
+    const int threads = 256;
+    const long long want = (rows * (D * 2 / 16) / 2 + threads - 1) / threads;
+    const long long cap = (long long)sm_count() * 8;
+    const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
+    cudaStream_t s = (cudaStream_t)stream;
+    if (D == 128)
+        permute3_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)q, (const uint4*)k,
+                                                      (const uint4*)v, (uint4*)q_out, (uint4*)k_out, (uint4*)v_out);
+    else
+        permute3_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)q, (const uint4*)k,
+                                                     (const uint4*)v, (uint4*)q_out, (uint4*)k_out, (uint4*)v_out);
+    return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }

@@ -241,6 +241,13 @@ int vsa_permute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* 
  * are dropped.  Asynchronous. */
 int vsa_unpermute(vsa_plan_t plan, const void* in, void* out, int B, int D, void* stream);
 
+/* q, k and v through the same permutation in one launch (the slot -> token
+ * arithmetic done once per row for the three tensors); same layouts,
+ * ownership and errors as vsa_permute, and no output may overlap an input or
+ * another output (VSA_ERR_INVALID_ARG). */
+int vsa_permute_qkv(vsa_plan_t plan, const void* q, const void* k, const void* v,
+                    void* q_out, void* k_out, void* v_out, int B, int D, void* stream);
+
 /* Block-sparse attention forward on tile-major tensors.
  * q, k, v: bf16 [B][num_heads][n_slots][D]; o: bf16 same shape;
  * lse: fp32 [B][num_heads][n_slots] (natural log of the sum over kept keys of

@@ -97,6 +97,7 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_svg_route(None, None, None, None, 1, 128, None, 1, 0.1, None, None, None, 0, None) == -1
     assert L.vsa_plan_apply_route(None, None, None) == -1
     assert L.vsa_ulysses_permute(None, None, 1, 128, 0, 1, None, None, None) == -1
+    assert L.vsa_permute_qkv(None, None, None, None, None, None, None, 1, 128, None) == -1
     assert L.vsa_ulysses_unpermute(None, None, 1, 128, 0, 1, None, None, None) == -1
 
 

@@ -133,6 +133,15 @@ def test_permute_bit_exact_and_round_trip(run):
     assert torch.equal(back.view(torch.int16), xd.view(torch.int16))
 
 
+def test_permute_qkv_matches_single_permutes(run):
+    import torch
+    import block_sparse_attention_mask_b200 as vsa
+    xs = [torch_bf16(x) for x in (run.q, run.k, run.v)]
+    fused = vsa.permute_qkv(run.plan, *xs)
+    for x, f in zip(xs, fused):
+        assert torch.equal(vsa.permute(run.plan, x).view(torch.int16), f.view(torch.int16))
+
+
 def test_attention_all_rows(run):
     w = run.w
     for h in range(w.heads):
