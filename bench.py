@@ -51,6 +51,7 @@ WORKLOADS = {
     "svg_wan720p_rounded": lambda: W.svg_wan720p(tile_round=1),
     "svg_wan720p_temporal_f0_rounded": lambda: W.svg_wan720p(temporal_layout=1, tile_round=1),
     "svg_wan720p_routing": W.svg_wan720p_routing,
+    "svg_wan720p_routing_f0": lambda: W.svg_wan720p_routing(temporal_layout=1),
     "tiny": W.tiny,
     "sta_hunyuan720p": W.sta_hunyuan720p,
     "stripe_wan720p": W.stripe_wan720p,

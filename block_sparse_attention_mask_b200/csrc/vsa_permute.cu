@@ -50,16 +50,30 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_ma
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
     const int sub = lane / VPR, v = lane % VPR;
     const int HW = d.H * d.W;
-    for (long long r = warp * RPW + sub; r < rows; r += nwarps * RPW) {
-        const long long bh = r / d.N;
-        const long long n = r - bh * d.N;
-        const int t = (int)(n / HW);
-        const int rem = (int)(n - (long long)t * HW);
-        const int h = rem / d.W, w = rem - (rem / d.W) * d.W;
-        const long long p = __ldg(&specs[bh % d.heads].layout) == VSA_LAYOUT_FRAME0_FIRST
-                                ? vsa_token_slot_f0(d, t, h, w)
-                                : vsa_token_slot(d, t, h, w);
-        out[r * VPR + v] = __ldg(in + (bh * d.Nslots + p) * VPR + v);
+    const long long stride = nwarps * RPW;
+    // two rows per thread in flight: both loads are issued before the stores
+    for (long long r0 = warp * RPW + sub; r0 < rows; r0 += 2 * stride) {
+        uint4 val[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const long long r = r0 + u * stride;
+            if (r < rows) {
+                const long long bh = r / d.N;
+                const long long n = r - bh * d.N;
+                const int t = (int)(n / HW);
+                const int rem = (int)(n - (long long)t * HW);
+                const int h = rem / d.W, w = rem - (rem / d.W) * d.W;
+                const long long p = __ldg(&specs[bh % d.heads].layout) == VSA_LAYOUT_FRAME0_FIRST
+                                        ? vsa_token_slot_f0(d, t, h, w)
+                                        : vsa_token_slot(d, t, h, w);
+                val[u] = __ldg(in + (bh * d.Nslots + p) * VPR + v);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const long long r = r0 + u * stride;
+            if (r < rows) out[r * VPR + v] = val[u];
+        }
     }
 }
 

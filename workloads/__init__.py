@@ -132,16 +132,19 @@ def svg_wan720p(temporal_layout: int = 0, tile_round: int = 0) -> Workload:
     return Workload(name, 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128, specs)
 
 
-def svg_wan720p_routing(amp: float = 10.0) -> Workload:
+def svg_wan720p_routing(amp: float = 10.0, temporal_layout: int = 0) -> Workload:
     """SVG routing on the Wan 720p latent: every head has both candidates
     (spatial |dt| <= 1 and temporal |dh| <= 5, |dw| <= 8, both with the
     frame-0 sink).  The q/k draws of heads 0-4 carry a per-frame embedding and
     those of heads 5-9 a per-position embedding, so that the former attend
     within their frame (spatial heads) and the latter to their position across
-    frames (temporal heads).  The plan starts with every head spatial."""
+    frames (temporal heads).  The plan starts with every head spatial.
+    temporal_layout=1 gives the temporal candidate the frame-0-first order,
+    which the routed heads then take."""
     sp = mask_spec("spatial", sink=1, rt=1)
-    tm = mask_spec("temporal", sink=1, rh=5, rw=8)
-    return Workload("svg_wan720p_routing_21x45x80", 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128,
+    tm = mask_spec("temporal", sink=1, rh=5, rw=8, layout=temporal_layout)
+    name = "svg_wan720p_routing_21x45x80" + ("_temporal_frame0_first" if temporal_layout else "")
+    return Workload(name, 1, 21, 45, 80, 10, 128, (1, 8, 16), 128, 128,
                     tuple([sp] * 10), structure=tuple(["frame"] * 5 + ["position"] * 5),
                     structure_amp=amp, route_specs=tuple([(sp, tm)] * 10))
 
