@@ -13,6 +13,12 @@ the attention kernel is also timed alone inside every step.
 Throughput is effective TFLOP/s over executed tiles: 4 * d * Bq * Bk FLOPs per
 full or boundary (q tile, kv tile) pair of the map, per head and batch.
 
+e2e: the same step from pinned host buffers through the host-buffer entry
+point (vsa_pipeline_run: per chunk of heads, the host-to-device copies of
+q, k, v, the step's kernels and the device-to-host copies of o and lse on
+three streams, overlapped), timed with CUDA events on the caller's stream.
+Routed workloads time it with the copies and the step in series.
+
 N > 1 (torchrun): each rank runs the same workload on its own GPU and its own
 batch element (weak scaling; heads and batches are independent, so there is
 no data-path collective).  Step times are the max over ranks.
@@ -44,6 +50,7 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES = {"plan_build": 3, "plan_build_stripe": 4, "permute": 1, "unpermute": 1, "fwd": 1,
             "route": 3, "apply": 1}
 ROUTE_FRAC = 0.01      # sampled share of the tokens for SVG routing
+E2E_CHUNK_HEADS = 1    # heads per chunk of the copy-overlapped host-buffer path
 
 WORKLOADS = {
     "svg_wan720p": W.svg_wan720p,
@@ -388,8 +395,17 @@ def run_gpu(args, w, world, rank, local):
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
     lse_host = torch.empty(lse.shape, dtype=torch.float32).pin_memory()
     qd, kd, vd = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    pipe = None
+    if not routed:
+        # the host-buffer entry point: copies overlapped with compute, one
+        # chunk of heads at a time (vsa_pipeline_run)
+        pipe = vsa.Pipeline(list(w.specs), grid, w.unit, w.q_tile, w.kv_tile, B=B, D=w.D,
+                            chunk_heads=E2E_CHUNK_HEADS)
 
     def e2e_step():
+        if pipe is not None:
+            pipe.run(pinned[0], pinned[1], pinned[2], o_host, lse_host, w.scale, sh)
+            return
         qd.copy_(pinned[0], non_blocking=True)
         kd.copy_(pinned[1], non_blocking=True)
         vd.copy_(pinned[2], non_blocking=True)
@@ -418,6 +434,9 @@ def run_gpu(args, w, world, rank, local):
     barrier(world)
     ms_e2e = max_over_ranks(statistics.mean([a.elapsed_time(b) for a, b in ev]), world, dev)
     plan.check(stream)
+    if pipe is not None:
+        pipe.check(stream)
+        pipe.close()
     h2d = 3 * q.numel() * 2
     d2h = o.numel() * 2 + lse.numel() * 4
 

@@ -88,6 +88,11 @@ def _load() -> ctypes.CDLL:
         "vsa_plan_apply_route": ([vp, vp, vp], i32),
         "vsa_ulysses_permute": ([vp, vp, i32, i32, i32, i32, vp, P(vp), vp], i32),
         "vsa_ulysses_unpermute": ([vp, vp, i32, i32, i32, i32, vp, P(vp), vp], i32),
+        "vsa_pipeline_create": ([P(vsa_mask_spec), i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i32, i32,
+                                 P(vp)], i32),
+        "vsa_pipeline_run": ([vp, vp, vp, vp, vp, vp, f32, vp], i32),
+        "vsa_pipeline_check_status": ([vp, vp], i32),
+        "vsa_pipeline_destroy": ([vp], i32),
         "vsa_status_string": ([i32], ctypes.c_char_p),
         "vsa_version": ([], i32),
     }
@@ -469,4 +474,39 @@ def svg_route(plan: Plan, q, k, v, rows, scale: Optional[float] = None, workspac
     vsa_svg_route(plan.handle, q, k, v, B, D, rows, R, scale, err, flags, workspace,
                   workspace.numel() * workspace.element_size(), stream)
     return err, flags
+
+
+class Pipeline:
+    """Attention from host buffers with the PCIe copies overlapped with the
+    compute, chunk by chunk of heads (see ``vsa_pipeline_run`` in
+    ``include/vsa.h``)."""
+
+    def __init__(self, specs: Sequence[Dict[str, int]], grid: Sequence[int], unit: Sequence[int],
+                 q_tile: int = 128, kv_tile: int = 128, B: int = 1, D: int = 128, chunk_heads: int = 1):
+        arr = (vsa_mask_spec * len(specs))(*[make_spec(d) for d in specs])
+        h = ctypes.c_void_p()
+        _check(_lib.vsa_pipeline_create(arr, len(specs), int(grid[0]), int(grid[1]), int(grid[2]),
+                                        int(unit[0]), int(unit[1]), int(unit[2]), q_tile, kv_tile, B, D,
+                                        chunk_heads, ctypes.byref(h)), "vsa_pipeline_create")
+        self.handle = h.value
+        self.B, self.D, self.heads = B, D, len(specs)
+
+    def run(self, q_host, k_host, v_host, o_host, lse_host, scale: float, stream=None) -> None:
+        """Host tensors (pinned): q, k, v, o bf16 [B, Hh, N, D]; lse fp32 [B, Hh, n_slots]."""
+        _check(_lib.vsa_pipeline_run(self.handle, _ptr(q_host), _ptr(k_host), _ptr(v_host), _ptr(o_host),
+                                     _ptr(lse_host), scale, _stream(stream)), "vsa_pipeline_run")
+
+    def check(self, stream=None) -> None:
+        _check(_lib.vsa_pipeline_check_status(self.handle, _stream(stream)), "vsa_pipeline_check_status")
+
+    def close(self) -> None:
+        if getattr(self, "handle", None):
+            _check(_lib.vsa_pipeline_destroy(self.handle), "vsa_pipeline_destroy")
+            self.handle = None
+
+    def __del__(self):  # pragma: no cover - best effort
+        try:
+            self.close()
+        except Exception:
+            pass
 

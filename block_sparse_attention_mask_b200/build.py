@@ -15,7 +15,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libvsa.so")
-SOURCES = ["vsa_plan.cu", "vsa_permute.cu", "vsa_attn.cu", "vsa_route.cu", "vsa_ulysses.cu", "vsa_api.cu", "vsa_noalloc.cu"]
+SOURCES = ["vsa_plan.cu", "vsa_permute.cu", "vsa_attn.cu", "vsa_route.cu", "vsa_ulysses.cu", "vsa_pipeline.cu", "vsa_api.cu", "vsa_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

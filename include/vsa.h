@@ -342,6 +342,37 @@ int vsa_ulysses_permute(vsa_plan_t plan, const void* x, int B, int D, int rank, 
 int vsa_ulysses_unpermute(vsa_plan_t plan, const void* o, int B, int D, int rank, int world,
                           const int32_t* head_layout, void* const* dst, void* stream);
 
+/* ---- Host buffers, copies overlapped with compute ------------------------
+ * The (batch, head) pairs are cut into chunks of chunk_heads heads, each with
+ * its own plan (the specs of those heads).  Per chunk, on three internal
+ * streams: host -> device copies of q, k, v; plan rebuild (first batch) +
+ * vsa_permute_qkv + vsa_sparse_attn_fwd + vsa_unpermute; device -> host
+ * copies of o and lse.  Two sets of device staging buffers alternate, so
+ * chunk c computes while chunk c+1's inputs and chunk c-1's outputs cross
+ * PCIe.
+ *
+ * vsa_pipeline_create: same spec / grid / tile arguments and errors as
+ * vsa_plan_create, plus B >= 1, D in {64,128}, chunk_heads >= 1; allocates
+ * the plans and 2 x chunk_heads x (4 natural + 4 tile-major) rows of
+ * staging on the current device.  Synchronous.
+ * vsa_pipeline_run: q, k, v, o host bf16 [B][num_heads][N][D] natural order,
+ * lse host fp32 [B][num_heads][n_slots] (tile-major, as vsa_sparse_attn_fwd);
+ * pinned (page-locked) memory for the copies to overlap.  Work starts after
+ * everything already on `stream` and `stream` resumes after the last copy
+ * back; nothing is synchronised on the host.  The host buffers must stay
+ * valid until then.
+ * vsa_pipeline_check_status: vsa_check_status over every chunk's plan.
+ * vsa_pipeline_destroy: synchronises the device, frees everything. */
+typedef struct vsa_pipeline_s* vsa_pipeline_t;
+int vsa_pipeline_create(const vsa_mask_spec* specs, int num_heads, int T, int H, int W,
+                        int bt, int bh, int bw, int q_tile, int kv_tile, int B, int D,
+                        int chunk_heads, vsa_pipeline_t* out);
+int vsa_pipeline_run(vsa_pipeline_t p, const void* q_host, const void* k_host,
+                     const void* v_host, void* o_host, float* lse_host, float scale,
+                     void* stream);
+int vsa_pipeline_check_status(vsa_pipeline_t p, void* stream);
+int vsa_pipeline_destroy(vsa_pipeline_t p);
+
 /* Synchronises `stream`, then reports and clears the plan's device status
  * word: VSA_OK, VSA_ERR_TIMEOUT or VSA_ERR_DEVICE; VSA_ERR_CUDA if the
  * stream itself failed. */

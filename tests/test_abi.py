@@ -98,6 +98,11 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_plan_apply_route(None, None, None) == -1
     assert L.vsa_ulysses_permute(None, None, 1, 128, 0, 1, None, None, None) == -1
     assert L.vsa_permute_qkv(None, None, None, None, None, None, None, 1, 128, None) == -1
+    assert L.vsa_pipeline_run(None, None, None, None, None, None, 0.1, None) == -1
+    assert L.vsa_pipeline_check_status(None, None) == -1
+    assert L.vsa_pipeline_destroy(None) == -1
+    h = ctypes.c_void_p()
+    assert L.vsa_pipeline_create(None, 1, 2, 2, 2, 1, 1, 1, 128, 128, 1, 128, 1, ctypes.byref(h)) == -1
     assert L.vsa_ulysses_unpermute(None, None, 1, 128, 0, 1, None, None, None) == -1
 
 
