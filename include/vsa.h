@@ -33,9 +33,12 @@
  * "aligning the sparse mask with execution").
  *
  * Memory.  The caller owns q, k, v, o and lse (device memory, contiguous,
- * 16-byte aligned).  A plan owns its device buffers and is immutable after
- * creation; vsa_plan_build may rewrite them in place.  vsa_permute,
- * vsa_unpermute and vsa_sparse_attn_fwd allocate nothing.
+ * 16-byte aligned).  A plan owns its device buffers; their shapes never
+ * change after creation.  vsa_plan_build rewrites the maps in place, and
+ * vsa_plan_apply_route rewrites the head specs on the device and then the
+ * maps.  vsa_permute, vsa_permute_qkv, vsa_unpermute, vsa_sparse_attn_fwd,
+ * vsa_svg_route (caller's workspace), vsa_plan_apply_route and the
+ * vsa_ulysses_* exchange allocate nothing.
  *
  * Streams.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
  * stream).  Every launch is asynchronous on that stream; host-visible results
