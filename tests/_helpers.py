@@ -31,7 +31,7 @@ def inverse_perm(perm: np.ndarray, n_tokens: int) -> np.ndarray:
     return inv
 
 
-class GpuRun:
+class PathRun:
     """Run the whole path (plan, permute, forward, unpermute) on one workload."""
 
     def __init__(self, w: W.Workload, inputs=None):

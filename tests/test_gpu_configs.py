@@ -11,7 +11,7 @@ import pytest
 
 import oracle
 import workloads as W
-from _helpers import GpuRun, oracle_map_rows, sample_qtiles
+from _helpers import PathRun, oracle_map_rows, sample_qtiles
 
 pytestmark = pytest.mark.gpu
 
@@ -27,7 +27,7 @@ def _inputs(w):
 
 
 def _check(w, heads, rows_per_head, map_heads, qtiles_per_head=6):
-    r = GpuRun(w, _inputs(w))
+    r = PathRun(w, _inputs(w))
     try:
         errs = []
         for h in heads:

@@ -10,7 +10,7 @@ import pytest
 
 import oracle
 import workloads as W
-from _helpers import GpuRun, torch_bf16
+from _helpers import PathRun, torch_bf16
 
 pytestmark = pytest.mark.gpu
 
@@ -76,7 +76,7 @@ def _workload(name):
 @pytest.fixture(scope="module", params=sorted(CASES))
 def run(request):
     w = _workload(request.param)
-    r = GpuRun(w)
+    r = PathRun(w)
     yield r
     r.close()
 

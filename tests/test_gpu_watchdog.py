@@ -7,7 +7,7 @@ import pytest
 
 import block_sparse_attention_mask_b200 as vsa
 import workloads as W
-from _helpers import GpuRun
+from _helpers import PathRun
 
 pytestmark = pytest.mark.gpu
 
@@ -25,7 +25,7 @@ def test_watchdog_reports_timeout_and_context_survives():
     plan.check()                                        # the status word was cleared
     plan.close()
     # the context still runs the real path correctly
-    r = GpuRun(w)
+    r = PathRun(w)
     for h in range(w.heads):
         r.check_rows(h, np.arange(w.N))
     r.close()
