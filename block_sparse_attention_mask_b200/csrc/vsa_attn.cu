@@ -88,7 +88,12 @@ struct Cfg {
     static constexpr int COL_S1 = BK;
     static constexpr int COL_O0 = 2 * BK;
     static constexpr int COL_O1 = 2 * BK + D;
-    static constexpr int COLS_USED = 2 * BK + 2 * D;
+    // Q also goes to TMEM (bf16 pairs, D/2 columns) when it fits: QK then
+    // reads only K from shared memory (the TS form), which keeps the
+    // half-width QK of 64-key tiles at the math rate
+    static constexpr bool Q_TMEM = 2 * BK + 2 * D + D / 2 <= 512;
+    static constexpr int COL_Q = 2 * BK + 2 * D;
+    static constexpr int COLS_USED = 2 * BK + 2 * D + (Q_TMEM ? D / 2 : 0);
     static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM budget");
     // shared memory map (offsets from a 1024-aligned base)
@@ -105,7 +110,7 @@ struct Cfg {
     static constexpr int OFF_BAR = OFF_ROWCTX + kRows * (int)sizeof(vsa_row_ctx);
     // barriers: k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], q_full,
     //           s_full[2], p_full[2], pv_done[2], mask_full[M], mask_empty[M], mma_drain
-    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 8 + 2 * kMaskSlots;
+    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 9 + 2 * kMaskSlots;
     // tmem addr, abort flag, and for the teardown after an abort: K and V
     // copies started, MMAs started (4 bytes each)
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
@@ -395,6 +400,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     auto BAR_MF = [&](int k) { return bar0 + 8u * (B1 + 7 + k); };
     auto BAR_ME = [&](int k) { return bar0 + 8u * (B1 + 7 + kMaskSlots + k); };
     const uint32_t BAR_DR = bar0 + 8u * (B1 + 7 + 2 * kMaskSlots);
+    const uint32_t BAR_QT = bar0 + 8u * (B1 + 8 + 2 * kMaskSlots);     // Q copied into TMEM
     uint32_t* maskbuf = (uint32_t*)(smem + C::OFF_MASK);
     float2* stat = (float2*)(smem + C::OFF_STAT);
     vsa_row_ctx* rowctx = (vsa_row_ctx*)(smem + C::OFF_ROWCTX);
@@ -419,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         }
         mbar_init(BAR_QF, 1);
         mbar_init(BAR_DR, 1);
+        mbar_init(BAR_QT, 4);                           // the four warps of softmax warpgroup 0
         for (int x = 0; x < 2; ++x) {
             mbar_init(BAR_SF(x), 1);
             mbar_init(BAR_PF(x), 4);                    // the four warps of softmax warpgroup x
@@ -483,7 +490,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         // added (the start-address field sits in the low bits and never carries).
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
         const uint32_t leader = elect_one();
-        if (cnt > 0 && mbar_wait_warp(BAR_QF, 0, ctl)) {
+        if (cnt > 0 && mbar_wait_warp(C::Q_TMEM ? BAR_QT : BAR_QF, 0, ctl)) {
             tc_fence_after();
             const uint64_t qdesc = smem_desc(s_base + C::OFF_Q, 16, 1024);
             const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
@@ -496,12 +503,22 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tc_fence_after();
                 const uint32_t dS = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
                 const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
-                mma_ss_lead<0>(dS, qdesc, kd, C::IDESC_QK, leader);
+                if constexpr (C::Q_TMEM) {
+                    // A = Q from TMEM: 16 elements of D per step are 8 columns
+                    mma_ts_lead<0>(dS, tmem + C::COL_Q, kd, C::IDESC_QK, leader);
 #pragma unroll
-                for (int kk = 1; kk < D / 16; ++kk)
-                    mma_ss_lead<1>(dS, qdesc + (uint64_t)((((kk >> 2) * (kRows * 128)) + (kk & 3) * 32) >> 4),
-                                   kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4), C::IDESC_QK,
-                                   leader);
+                    for (int kk = 1; kk < D / 16; ++kk)
+                        mma_ts_lead<1>(dS, tmem + C::COL_Q + kk * 8,
+                                       kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
+                                       C::IDESC_QK, leader);
+                } else {
+                    mma_ss_lead<0>(dS, qdesc, kd, C::IDESC_QK, leader);
+#pragma unroll
+                    for (int kk = 1; kk < D / 16; ++kk)
+                        mma_ss_lead<1>(dS, qdesc + (uint64_t)((((kk >> 2) * (kRows * 128)) + (kk & 3) * 32) >> 4),
+                                       kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4),
+                                       C::IDESC_QK, leader);
+                }
                 tc_commit_lead(BAR_SF(j & 1), leader);
                 tc_commit_lead(BAR_KE(st), leader);
                 return true;
@@ -599,6 +616,34 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
+        if constexpr (C::Q_TMEM) {
+            // warpgroup 0 moves Q into TMEM: thread r reads row r from the
+            // 128-byte-swizzled shared copy (chunk u of a 64-column block at
+            // u ^ (r mod 8)) and stores it as bf16 pairs, row r = lane r
+            if (X == 0 && cnt > 0) {
+                ok = mbar_wait_warp(BAR_QF, 0, ctl);
+                if (ok) {
+#pragma unroll
+                    for (int c = 0; c < D / 64; ++c) {
+                        uint32_t qv[32];
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            const uint4 v4 = *reinterpret_cast<const uint4*>(
+                                smem + C::OFF_Q + c * (kRows * 128) + row * 128 + ((u ^ (row & 7)) << 4));
+                            qv[4 * u] = v4.x;
+                            qv[4 * u + 1] = v4.y;
+                            qv[4 * u + 2] = v4.z;
+                            qv[4 * u + 3] = v4.w;
+                        }
+                        tmem_st32(tmem + lane_off + C::COL_Q + c * 32, qv);
+                    }
+                    tmem_st_wait();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(BAR_QT);
+                }
+            }
+        }
         int ent_next = cnt > 0 ? __ldg(entries) : 0;
         int kb = 0;                                       // boundary tiles of the list so far
         for (int j = 0; j < cnt && ok; ++j) {
