@@ -83,3 +83,89 @@ def test_random_tile_maps_and_rows(i):
             err = np.abs(o[0, h][rows] - ref)
             assert err.max() <= TOL_MAX and err.mean() <= TOL_MEAN, (i, h, spec, err.max(), err.mean())
     plan.close()
+
+
+def _route_cases(n, seed):
+    g = np.random.Generator(np.random.PCG64(seed))
+    out = []
+    for _ in range(n):
+        T, H, Wd = int(g.integers(1, 6)), int(g.integers(1, 12)), int(g.integers(1, 20))
+        heads = int(g.integers(1, 4))
+        sp = [S("spatial", int(g.integers(0, 2)), rt=int(g.integers(0, T))) for _ in range(heads)]
+        tm = [S("temporal", int(g.integers(0, 2)), rh=int(g.integers(0, H)), rw=int(g.integers(0, Wd)),
+                layout=int(g.integers(0, 2))) for _ in range(heads)]
+        structure = tuple(["", "frame", "position"][int(g.integers(0, 3))] for _ in range(heads))
+        out.append(((T, H, Wd), heads, int(g.choice([64, 128])), int(g.integers(1, 3)), sp, tm, structure,
+                    float(g.uniform(0.02, 1.0))))
+    return out
+
+
+ROUTE_CASES = _route_cases(40, 77)
+
+
+@pytest.mark.parametrize("i", range(len(ROUTE_CASES)))
+def test_random_routing(i):
+    import torch
+    import block_sparse_attention_mask_b200 as vsa
+    grid, heads, D, B, sp, tm, structure, frac = ROUTE_CASES[i]
+    T, H, Wd = grid
+    w = W.Workload(f"route_fuzz_{i}", B, T, H, Wd, heads, D, (1, 8, 16), 128, 128, tuple(sp),
+                   structure=structure, structure_amp=6.0, route_specs=tuple(zip(sp, tm)))
+    x = [W.full_tensor(w, c) for c in "qkv"]
+    rows = W.route_rows(w.N, frac, seed=i)
+    plan = vsa.Plan(list(sp), grid, w.unit, 128, 128)
+    plan.set_route_candidates(sp, tm)
+    err, flags = vsa.svg_route(plan, *(torch_bf16(t) for t in x),
+                               torch.as_tensor(rows.astype(np.int32)).cuda(), scale=w.scale)
+    torch.cuda.synchronize()
+    plan.check()
+    err_g, flags_g = err.cpu().numpy().astype(np.float64), flags.cpu().numpy()
+    err_o, flags_o = oracle.svg_route(sp, tm, grid, D, w.scale, *x, rows)
+    eps = 5e-3
+    tol = 2.0 * np.sqrt(err_o) * eps + eps * eps
+    assert np.all(np.abs(err_g - err_o) <= tol), (i, err_g, err_o)
+    assert np.array_equal(flags_g, (err_g[:, 1] < err_g[:, 0]).astype(flags_g.dtype))
+    decisive = np.abs(err_o[:, 0] - err_o[:, 1]) > tol[:, 0] + tol[:, 1]
+    assert np.array_equal(flags_g[decisive], flags_o[decisive]), (i, flags_g, flags_o)
+    plan.close()
+
+
+@pytest.mark.parametrize("seed", range(12))
+def test_random_exchange(seed):
+    import torch
+    import block_sparse_attention_mask_b200 as vsa
+    g = np.random.Generator(np.random.PCG64(1000 + seed))
+    world = int(g.integers(1, 9))
+    hpr = int(g.integers(1, 3))
+    grid = (int(g.integers(1, 5)), int(g.integers(1, 17)), int(g.integers(1, 21)))
+    N = int(np.prod(grid))
+    if N < world:
+        grid = (world, grid[1], grid[2])
+        N = int(np.prod(grid))
+    D, B = int(g.choice([64, 128])), int(g.integers(1, 3))
+    specs = [_random_spec(g, *grid) for _ in range(world * hpr)]
+    unit = (1, 8, 8)
+    plans = [vsa.Plan(specs[r * hpr:(r + 1) * hpr], grid, unit, 128, 128) for r in range(world)]
+    n_slots = plans[0].n_slots
+    layout = torch.tensor([s["layout"] for s in specs], dtype=torch.int32, device="cuda")
+    perms = [oracle.tile_major_order(grid, unit, n_slots, layout=s["layout"]) for s in specs]
+    x = W.bf16_bits_from_f32(g.standard_normal((B, world * hpr, N, D), dtype=np.float32))
+    shards, head_local = oracle.ulysses_exchange(x, world)
+    dst = [torch.full((B, hpr, n_slots, D), 3.0, dtype=torch.bfloat16, device="cuda") for _ in range(world)]
+    for r in range(world):
+        vsa.vsa_ulysses_permute(plans[r].handle, torch_bf16(shards[r]), B, D, r, world, layout, dst)
+    torch.cuda.synchronize()
+    for r in range(world):
+        want = oracle.layout_gather(head_local[r], perms[r * hpr:(r + 1) * hpr])
+        assert np.array_equal(dst[r].cpu().view(torch.int16).numpy().view(np.uint16), want), (seed, r)
+    off = oracle.shard_offsets(N, world)
+    outs = [torch.full((B, off[r + 1] - off[r], world * hpr, D), 3.0, dtype=torch.bfloat16, device="cuda")
+            for r in range(world)]
+    for r in range(world):
+        vsa.vsa_ulysses_unpermute(plans[r].handle, dst[r], B, D, r, world, layout, outs)
+    torch.cuda.synchronize()
+    # the round trip returns every shard unchanged
+    for r in range(world):
+        assert np.array_equal(outs[r].cpu().view(torch.int16).numpy().view(np.uint16), shards[r]), (seed, r)
+    for p in plans:
+        p.close()
