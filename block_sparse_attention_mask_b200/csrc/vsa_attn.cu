@@ -93,7 +93,7 @@ struct Cfg {
     // half-width QK of 64-key tiles at the math rate
     static constexpr bool Q_TMEM = 2 * BK + 2 * D + D / 2 <= 512;
     static constexpr int COL_Q = 2 * BK + 2 * D;
-    static constexpr int COLS_USED = 2 * BK + 2 * D + (Q_TMEM ? D / 2 : 0);
+    static constexpr int COLS_USED = COL_Q + (Q_TMEM ? D / 2 : 0);
     static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
     static_assert(COLS_USED <= 512, "TMEM budget");
     // shared memory map (offsets from a 1024-aligned base)
