@@ -51,6 +51,8 @@ struct vsa_plan_s {
     int has_stripe;
     vsa_mask_spec* d_cand;      // [2][heads] SVG routing candidates: spatial, temporal
     int has_cand;
+    int32_t* d_slot2tok;        // [2 layouts][Nslots] natural token of a slot, -1 for padding
+    int32_t* d_tok2slot;        // [2 layouts][N] slot of a natural token
 };
 
 // Host helpers ------------------------------------------------------------

@@ -4,7 +4,9 @@
 // [N, d] gather; "Parameterized Stripe Attention", key design 2: hierarchical
 // layout with 3D padding), or the frame-0-first position-major order of
 // temporal heads ("Sparse VideoGen: accelerating video diffusion attention on
-// TPU", "arranging tokens for efficient temporal access").  HBM-bound copies: every row of D bf16 values moves as 16-byte
+// TPU", "arranging tokens for efficient temporal access").  HBM-bound copies: the
+// plan's lookup tables give each slot's token (and each token's slot) in both
+// orders, and every row of D bf16 values moves as 16-byte
 // vectors, a warp covers 2 rows (D = 128) or 4 rows (D = 64) per step, and
 // the grid is a multiple of the SM count with a grid-stride loop.
 #include <cuda_runtime.h>
@@ -15,8 +17,8 @@ namespace {
 
 template <int D>
 __global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
-                                                      long long rows, const uint4* __restrict__ in,
-                                                      uint4* __restrict__ out)
+                                                      const int32_t* __restrict__ s2t, long long rows,
+                                                      const uint4* __restrict__ in, uint4* __restrict__ out)
 {
     constexpr int VPR = D * 2 / 16;   // 16-byte vectors per row
     constexpr int RPW = 32 / VPR;     // rows per warp step
@@ -27,21 +29,16 @@ __global__ void __launch_bounds__(256) permute_kernel(vsa_dims d, const vsa_mask
     for (long long r = warp * RPW + sub; r < rows; r += nwarps * RPW) {
         const long long bh = r / d.Nslots;
         const long long p = r - bh * d.Nslots;
-        int t = 0, h = 0, w = 0;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
         const int layout = __ldg(&specs[bh % d.heads].layout);
-        if (vsa_slot_coords_any(d, layout, p, t, h, w)) {
-            const long long n = ((long long)t * d.H + h) * d.W + w;
-            val = __ldg(in + (bh * d.N + n) * VPR + v);
-        }
-        out[r * VPR + v] = val;
+        const int n = __ldg(s2t + layout * d.Nslots + p);
+        out[r * VPR + v] = n >= 0 ? __ldg(in + (bh * d.N + n) * VPR + v) : make_uint4(0u, 0u, 0u, 0u);
     }
 }
 
 template <int D>
 __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
-                                                        long long rows, const uint4* __restrict__ in,
-                                                        uint4* __restrict__ out)
+                                                        const int32_t* __restrict__ t2s, long long rows,
+                                                        const uint4* __restrict__ in, uint4* __restrict__ out)
 {
     constexpr int VPR = D * 2 / 16;
     constexpr int RPW = 32 / VPR;
@@ -49,7 +46,6 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_ma
     const long long warp = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
     const int sub = lane / VPR, v = lane % VPR;
-    const int HW = d.H * d.W;
     const long long stride = nwarps * RPW;
     // two rows per thread in flight: both loads are issued before the stores
     for (long long r0 = warp * RPW + sub; r0 < rows; r0 += 2 * stride) {
@@ -60,12 +56,8 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_ma
             if (r < rows) {
                 const long long bh = r / d.N;
                 const long long n = r - bh * d.N;
-                const int t = (int)(n / HW);
-                const int rem = (int)(n - (long long)t * HW);
-                const int h = rem / d.W, w = rem - (rem / d.W) * d.W;
-                const long long p = __ldg(&specs[bh % d.heads].layout) == VSA_LAYOUT_FRAME0_FIRST
-                                        ? vsa_token_slot_f0(d, t, h, w)
-                                        : vsa_token_slot(d, t, h, w);
+                const int layout = __ldg(&specs[bh % d.heads].layout);
+                const long long p = __ldg(t2s + layout * d.N + n);
                 val[u] = __ldg(in + (bh * d.Nslots + p) * VPR + v);
             }
         }
@@ -77,11 +69,12 @@ __global__ void __launch_bounds__(256) unpermute_kernel(vsa_dims d, const vsa_ma
     }
 }
 
-// q, k and v in one pass: the slot -> token arithmetic is done once per row
-// for the three tensors, and each thread keeps six 16-byte loads (two rows
-// of each tensor) in flight before its stores.
+// q, k and v in one pass: one slot -> token lookup per row serves the three
+// tensors, and each thread keeps six 16-byte loads (two rows of each tensor)
+// in flight before its stores.
 template <int D>
 __global__ void __launch_bounds__(256) permute3_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs,
+                                                       const int32_t* __restrict__ s2t,
                                                        long long rows, const uint4* __restrict__ q,
                                                        const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                        uint4* __restrict__ qo, uint4* __restrict__ ko,
@@ -105,11 +98,11 @@ __global__ void __launch_bounds__(256) permute3_kernel(vsa_dims d, const vsa_mas
             if (r < rows) {
                 const long long bh = r / d.Nslots;
                 const long long p = r - bh * d.Nslots;
-                int t = 0, h = 0, w = 0;
                 const int layout = __ldg(&specs[bh % d.heads].layout);
-                if (vsa_slot_coords_any(d, layout, p, t, h, w)) {
+                const int n = __ldg(s2t + layout * d.Nslots + p);
+                if (n >= 0) {
                     real[u] = true;
-                    src[u] = (bh * d.N + ((long long)t * d.H + h) * d.W + w) * VPR + c;
+                    src[u] = (bh * d.N + n) * VPR + c;
                 }
             }
         }
@@ -165,11 +158,11 @@ int launch(bool forward, vsa_plan_t plan, const void* in, void* out, int B, int 
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     cudaStream_t s = (cudaStream_t)stream;
     if (forward) {
-        if (D == 128) permute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
-        else permute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
+        if (D == 128) permute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_slot2tok, rows, (const uint4*)in, (uint4*)out);
+        else permute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_slot2tok, rows, (const uint4*)in, (uint4*)out);
     } else {
-        if (D == 128) unpermute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
-        else unpermute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)in, (uint4*)out);
+        if (D == 128) unpermute_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_tok2slot, rows, (const uint4*)in, (uint4*)out);
+        else unpermute_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_tok2slot, rows, (const uint4*)in, (uint4*)out);
     }
     return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
@@ -219,10 +212,10 @@ extern "C" int vsa_permute_qkv(vsa_plan_t plan, const void* q, const void* k, co
     const unsigned grid = (unsigned)(want < cap ? (want > 0 ? want : 1) : cap);
     cudaStream_t s = (cudaStream_t)stream;
     if (D == 128)
-        permute3_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)q, (const uint4*)k,
+        permute3_kernel<128><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_slot2tok, rows, (const uint4*)q, (const uint4*)k,
                                                       (const uint4*)v, (uint4*)q_out, (uint4*)k_out, (uint4*)v_out);
     else
-        permute3_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, rows, (const uint4*)q, (const uint4*)k,
+        permute3_kernel<64><<<grid, threads, 0, s>>>(d, plan->d_specs, plan->d_slot2tok, rows, (const uint4*)q, (const uint4*)k,
                                                      (const uint4*)v, (uint4*)q_out, (uint4*)k_out, (uint4*)v_out);
     return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }

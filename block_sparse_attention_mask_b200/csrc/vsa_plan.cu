@@ -501,6 +501,20 @@ __global__ void perm_kernel(vsa_dims d, int layout, int32_t* __restrict__ perm)
     perm[p] = vsa_slot_coords_any(d, layout, p, t, h, w) ? (int32_t)(((long long)t * d.H + h) * d.W + w) : -1;
 }
 
+// Both token orders as lookup tables: slot -> natural token and back.
+__global__ void order_tables_kernel(vsa_dims d, int32_t* __restrict__ s2t, int32_t* __restrict__ t2s)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const int layout = blockIdx.y;
+    if (i < d.Nslots) {
+        int t, h, w;
+        const bool real = vsa_slot_coords_any(d, layout, i, t, h, w);
+        const long long n = ((long long)t * d.H + h) * d.W + w;
+        s2t[layout * d.Nslots + i] = real ? (int32_t)n : -1;
+        if (real) t2s[layout * d.N + n] = (int32_t)i;
+    }
+}
+
 bool tile_fits_unit(int B, int U, int bh, int bw)
 {
     if (B >= U) return B % U == 0;
@@ -582,6 +596,8 @@ static void free_plan(vsa_plan_s* p)
     cudaFree(p->d_steps);
     cudaFree(p->d_status);
     cudaFree(p->d_cand);
+    cudaFree(p->d_slot2tok);
+    cudaFree(p->d_tok2slot);
     delete p;
 }
 
@@ -686,6 +702,8 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     ok = ok && cudaMalloc(&p->d_counts, sizeof(unsigned long long) * 3 * num_heads) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_steps, sizeof(unsigned long long) * num_heads) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_status, sizeof(unsigned int)) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_slot2tok, sizeof(int32_t) * 2 * (size_t)d.Nslots) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_tok2slot, sizeof(int32_t) * 2 * (size_t)d.N) == cudaSuccess;
     if (!ok) {
         cudaGetLastError();
         free_plan(p);
@@ -700,6 +718,11 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     }
     // the host copy of specs may be released as soon as the copy is done
     if (cudaStreamSynchronize(s) != cudaSuccess) {
+        free_plan(p);
+        return VSA_ERR_CUDA;
+    }
+    order_tables_kernel<<<dim3(blocks_for(d.Nslots, 256), 2), 256, 0, s>>>(d, p->d_slot2tok, p->d_tok2slot);
+    if (cudaGetLastError() != cudaSuccess) {
         free_plan(p);
         return VSA_ERR_CUDA;
     }
