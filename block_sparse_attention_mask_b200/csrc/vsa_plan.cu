@@ -36,12 +36,12 @@ struct Box {
 // real token.  Sets *pad when the tile holds any padding slot.
 __device__ bool tile_box(const vsa_dims& d, int tile, int B, int i, Box& bx, bool& pad)
 {
-    const long long p0 = (long long)tile * B;
+    const int p0 = tile * B;                 // < 2^24 + B: n_slots is capped at 2^24
     int u, t0, t1, h0, h1, w0, w1;
     if (B <= d.U) {
         if (p0 >= d.Npad) { pad = true; return false; }
-        u = (int)(p0 / d.U);
-        const int o0 = (int)(p0 - (long long)u * d.U);
+        u = p0 / d.U;
+        const int o0 = p0 - u * d.U;
         const int per_t = d.nTh * d.nTw;
         const int tt = u / per_t, th = (u - tt * per_t) / d.nTw, tw = u - tt * per_t - th * d.nTw;
         const int hw = d.bh * d.bw;
@@ -288,9 +288,19 @@ __global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ sp
     const long long per_head = (long long)d.nQ * d.nK;
     const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
     if (idx >= per_head * d.heads) return;
-    const int head = (int)(idx / per_head);
-    const long long rem = idx - (long long)head * per_head;
-    const int a = (int)(rem / d.nK), b = (int)(rem - (long long)a * d.nK);
+    int head, a, b;
+    if (per_head * d.heads <= 0x7FFFFFFFLL) {          // 32-bit division (the usual case)
+        const int i32 = (int)idx, ph = (int)per_head;
+        head = i32 / ph;
+        const int r = i32 - head * ph;
+        a = r / d.nK;
+        b = r - a * d.nK;
+    } else {
+        head = (int)(idx / per_head);
+        const long long rem = idx - (long long)head * per_head;
+        a = (int)(rem / d.nK);
+        b = (int)(rem - (long long)a * d.nK);
+    }
     const vsa_mask_spec m = specs[head];
     const uint32_t* sb = sbits ? sbits + (size_t)head * d.sbits_words : nullptr;
     if (m.layout == VSA_LAYOUT_FRAME0_FIRST) {
