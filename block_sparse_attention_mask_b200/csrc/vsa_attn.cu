@@ -497,9 +497,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
             const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
             constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
             // S_j = Q K_j^T into S_{j mod 2}; K_j's stage is released when it completes
-            auto issue_qk = [&](int j) -> bool {
+            auto issue_qk = [&](int j, bool waited) -> bool {
                 const int st = j % C::STAGES_K;
-                if (!mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES_K) & 1, ctl)) return false;
+                if (!waited && !mbar_wait_warp(BAR_KF(st), (uint32_t)(j / C::STAGES_K) & 1, ctl)) return false;
                 tc_fence_after();
                 const uint32_t dS = tmem + ((j & 1) ? C::COL_S1 : C::COL_S0);
                 const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
@@ -523,13 +523,18 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tc_commit_lead(BAR_KE(st), leader);
                 return true;
             };
-            bool go = issue_qk(0);
+            bool go = issue_qk(0, false);
             if (go && leader) issued[2] = 1;
-            go = go && (cnt < 2 || issue_qk(1));
+            go = go && (cnt < 2 || issue_qk(1, false));
             for (int j = 0; go && j < cnt; ++j) {
                 const int x = j & 1, vs = j % C::STAGES_V;
-                if (!mbar_wait_warp(BAR_PF(x), (uint32_t)(j >> 1) & 1, ctl)) break;
+                // V_j and K_{j+2} have usually landed long before P_j: wait for
+                // them first, so only the MMAs follow P_j's arrival
                 if (!mbar_wait_warp(BAR_VF(vs), (uint32_t)(j / C::STAGES_V) & 1, ctl)) break;
+                if (j + 2 < cnt &&
+                    !mbar_wait_warp(BAR_KF((j + 2) % C::STAGES_K), (uint32_t)((j + 2) / C::STAGES_K) & 1, ctl))
+                    break;
+                if (!mbar_wait_warp(BAR_PF(x), (uint32_t)(j >> 1) & 1, ctl)) break;
                 tc_fence_after();
                 // O_x (+)= P_j V_j, P_j in the first BK/2 columns of S_x
                 const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
@@ -543,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 tc_commit_lead(BAR_PV(x), leader);
                 tc_commit_lead(BAR_VE(vs), leader);
                 // S_{j+2} reuses S_x: queued behind PV_j, so P_j is read first
-                if (j + 2 < cnt) go = issue_qk(j + 2);
+                if (j + 2 < cnt) go = issue_qk(j + 2, true);
             }
         }
     } else if (warp >= kMaskWarp0) {
@@ -703,12 +708,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 }
             }
 
-            uint32_t pk[BK / 2];
             bool need_o = false;
             float alpha = 1.0f;
             if (cls == VSA_TILE_EMPTY) {
+                uint32_t zero[16];
 #pragma unroll
-                for (int c = 0; c < BK / 2; ++c) pk[c] = 0u;
+                for (int c = 0; c < 16; ++c) zero[c] = 0u;
+#pragma unroll
+                for (int q = 0; q < BK / 32; ++q) tmem_st16(tS + 16 * q, zero);
             } else {
                 // row max: independent chains of 3-input max over 32 columns each
                 float mc[BK / 32];
@@ -737,13 +744,19 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                 const unsigned long long mneg2 = f2_pack(mneg, mneg);
                 unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-                for (int i = 0; i < BK / 2; ++i) {
-                    float x0, x1;
-                    f2_unpack(f2_fma(f2_pack(s[2 * i], s[2 * i + 1]), sl2, mneg2), x0, x1);
-                    const float p0 = ex2(x0);
-                    const float p1 = ex2(x1);
-                    acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
-                    pk[i] = pack_bf16(p0, p1);
+                for (int q = 0; q < BK / 32; ++q) {
+                    uint32_t pq[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int c = 32 * q + 2 * i;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2, mneg2), x0, x1);
+                        const float p0 = ex2(x0);
+                        const float p1 = ex2(x1);
+                        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+                        pq[i] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tS + 16 * q, pq);
                 }
                 float a0, a1, a2, a3, a4, a5, a6, a7;
                 f2_unpack(acc[0], a0, a1);
@@ -768,9 +781,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
                     tmem_st32(tO + c * 32, ov);
                 }
             }
-            // P_j (bf16 pairs) over the first BK/2 columns of S_X
-#pragma unroll
-            for (int c = 0; c < BK / 64; ++c) tmem_st32(tS + c * 32, pk + c * 32);
+            // P_j went over the first BK/2 columns of S_X 32 keys at a time, each
+            // chunk stored as soon as its exponentials are done (fewer live
+            // registers than holding all of P_j); one wait covers them all
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
