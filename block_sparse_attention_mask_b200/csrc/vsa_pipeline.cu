@@ -7,6 +7,12 @@
 // every reuse.  The kernels are the plan's own: each chunk of heads has its
 // own plan (the specs of those heads), and its tensors are contiguous slices
 // of the [B][heads][...] host arrays.
+//
+// Chunks run in decreasing order of executed tile steps.  Every chunk of a
+// full size moves the same bytes over PCIe, so with copy-in and compute as a
+// two-stage flow shop, heaviest compute first is Johnson's rule: the chunks
+// whose compute outlasts their copy go while later copies are still coming,
+// and the chunk left to compute after the last copy is the lightest.
 #include <cuda_runtime.h>
 
 #include <cstring>
@@ -34,6 +40,7 @@ struct vsa_pipeline_s {
     long long N, Nslots;
     vsa_plan_t* plans;        // one per head chunk
     int* chunk_heads;         // heads in each head chunk
+    int* order;               // head chunks in issue order
     Staging set[kSets];
     cudaStream_t s_h2d, s_comp, s_d2h;
     cudaEvent_t start, done;
@@ -65,6 +72,7 @@ void destroy_pipeline(vsa_pipeline_s* p)
             if (p->plans[c]) vsa_plan_destroy(p->plans[c]);
     delete[] p->plans;
     delete[] p->chunk_heads;
+    delete[] p->order;
     if (p->s_h2d) cudaStreamDestroy(p->s_h2d);
     if (p->s_comp) cudaStreamDestroy(p->s_comp);
     if (p->s_d2h) cudaStreamDestroy(p->s_d2h);
@@ -97,7 +105,12 @@ extern "C" int vsa_pipeline_create(const vsa_mask_spec* specs, int num_heads, in
     }
     p->plans = new (std::nothrow) vsa_plan_t[p->nchunks_h]();
     p->chunk_heads = new (std::nothrow) int[p->nchunks_h]();
-    if (!p->plans || !p->chunk_heads) {
+    p->order = new (std::nothrow) int[p->nchunks_h]();
+    long long* work = new (std::nothrow) long long[p->nchunks_h]();
+    int64_t* steps = new (std::nothrow) int64_t[p->chunk]();
+    if (!p->plans || !p->chunk_heads || !p->order || !work || !steps) {
+        delete[] work;
+        delete[] steps;
         destroy_pipeline(p);
         return VSA_ERR_OOM;
     }
@@ -105,12 +118,25 @@ extern "C" int vsa_pipeline_create(const vsa_mask_spec* specs, int num_heads, in
         const int h0 = c * p->chunk;
         const int nh = (h0 + p->chunk <= num_heads) ? p->chunk : num_heads - h0;
         p->chunk_heads[c] = nh;
-        const int r = vsa_plan_create(specs + h0, nh, T, H, W, bt, bh, bw, q_tile, kv_tile, nullptr, &p->plans[c]);
+        int r = vsa_plan_create(specs + h0, nh, T, H, W, bt, bh, bw, q_tile, kv_tile, nullptr, &p->plans[c]);
+        if (r == VSA_OK) r = vsa_plan_exec_steps(p->plans[c], steps, (size_t)nh, nullptr);
         if (r != VSA_OK) {
+            delete[] work;
+            delete[] steps;
             destroy_pipeline(p);
             return r;
         }
+        for (int i = 0; i < nh; ++i) work[c] += steps[i];
+        // insertion by decreasing work; equal work keeps head order
+        int at = c;
+        while (at > 0 && work[p->order[at - 1]] < work[c]) {
+            p->order[at] = p->order[at - 1];
+            --at;
+        }
+        p->order[at] = c;
     }
+    delete[] work;
+    delete[] steps;
     p->N = p->plans[0]->d.N;
     p->Nslots = p->plans[0]->d.Nslots;
     const size_t nat = (size_t)p->chunk * p->N * D * 2, tm = (size_t)p->chunk * p->Nslots * D * 2;
@@ -164,7 +190,8 @@ extern "C" int vsa_pipeline_run(vsa_pipeline_t p, const void* q_host, const void
     VSA_CUDA_TRY(cudaStreamWaitEvent(p->s_d2h, p->start, 0));
     int c = 0;
     for (int b = 0; b < p->B; ++b)
-        for (int hc = 0; hc < p->nchunks_h; ++hc, ++c) {
+        for (int i = 0; i < p->nchunks_h; ++i, ++c) {
+            const int hc = p->order[i];
             Staging& st = p->set[c % kSets];
             vsa_plan_t plan = p->plans[hc];
             const int nh = p->chunk_heads[hc];

@@ -381,6 +381,116 @@ __global__ void tile_map_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ sp
     map[idx] = cls;
 }
 
+// The real boxes of one tile under one token order and its padding flag (any
+// slot of the tile that holds no real token).  Returns the number of boxes;
+// callers only use this where a tile has at most kMaxTileBoxes of them (a
+// frame-0-first tile always does; a tile-major tile when it spans at most
+// eight units).
+constexpr int kMaxTileBoxes = 8;
+
+__device__ int tile_boxes(const vsa_dims& d, int layout, int tile, int B, Box* bx, bool& pad)
+{
+    pad = false;
+    if (layout == VSA_LAYOUT_FRAME0_FIRST) return f0_tile_boxes(d, (long long)tile * B, B, bx, pad);
+    const int nb = B <= d.U ? 1 : B / d.U;
+    int n = 0;
+    for (int i = 0; i < nb && i < kMaxTileBoxes; ++i) {
+        Box b;
+        if (tile_box(d, tile, B, i, b, pad)) bx[n++] = b;
+    }
+    return n;
+}
+
+// Tile boxes kept in shared memory as int16 coordinates (T, H, W < 2^15),
+// field-major so that thread c reads column c without bank conflicts.
+template <int N>
+struct BoxCols {
+    short v[kMaxTileBoxes][6][N];
+    __device__ __forceinline__ void put(int j, int c, const Box& b)
+    {
+        v[j][0][c] = (short)b.t0; v[j][1][c] = (short)b.t1;
+        v[j][2][c] = (short)b.h0; v[j][3][c] = (short)b.h1;
+        v[j][4][c] = (short)b.w0; v[j][5][c] = (short)b.w1;
+    }
+    __device__ __forceinline__ Box get(int j, int c) const
+    {
+        return Box{v[j][0][c], v[j][1][c], v[j][2][c], v[j][3][c], v[j][4][c], v[j][5][c]};
+    }
+};
+
+constexpr int kMapKB = 128;  // kv tiles per block, one per thread
+constexpr int kMapQB = 32;   // q tiles per block
+
+// The tile map for tiles of at most kMaxTileBoxes boxes: one block per
+// (head, 32 q tiles, 128 kv tiles).  Each tile's boxes are derived once per
+// block into shared memory; a thread then classifies its kv tile against the
+// block's 32 q tiles (coalesced byte stores along kv).  Same classes as
+// tile_map_kernel below: any / all kept over the real (A x B) box pairs, or
+// the kept fraction under tile-aligned rounding.
+__global__ void __launch_bounds__(kMapKB) tile_map_blocked_kernel(vsa_dims d,
+                                                                  const vsa_mask_spec* __restrict__ specs,
+                                                                  const uint32_t* __restrict__ sbits,
+                                                                  int8_t* __restrict__ map)
+{
+    __shared__ BoxCols<kMapQB> qbx;
+    __shared__ BoxCols<kMapKB> kbx;
+    __shared__ unsigned char qn[kMapQB];
+    const int head = blockIdx.z;
+    const vsa_mask_spec m = specs[head];
+    const uint32_t* sb = sbits ? sbits + (size_t)head * d.sbits_words : nullptr;
+    const int c = threadIdx.x;
+    const int a0 = blockIdx.y * kMapQB;
+    const int b = blockIdx.x * kMapKB + c;
+    Box tmp[kMaxTileBoxes];
+    if (c < kMapQB) {
+        bool qpad;
+        const int n = (a0 + c < d.nQ) ? tile_boxes(d, m.layout, a0 + c, d.Bq, tmp, qpad) : 0;
+        for (int i = 0; i < n; ++i) qbx.put(i, c, tmp[i]);
+        qn[c] = (unsigned char)n;
+    }
+    bool kpad = false;
+    int nk = 0;
+    long long nkr = 0;
+    if (b < d.nK) {
+        nk = tile_boxes(d, m.layout, b, d.Bk, tmp, kpad);
+        for (int j = 0; j < nk; ++j) {
+            kbx.put(j, c, tmp[j]);
+            nkr += box_size(tmp[j]);
+        }
+    }
+    __syncthreads();
+    if (b >= d.nK) return;
+    const int na = min(kMapQB, d.nQ - a0);
+    int8_t* out = map + ((long long)head * d.nQ + a0) * d.nK + b;
+    for (int qi = 0; qi < na; ++qi, out += d.nK) {
+        const int nq = qn[qi];
+        int8_t cls;
+        if (m.tile_round) {
+            long long kept = 0, nqr = 0;
+            for (int i = 0; i < nq; ++i) {
+                const Box A = qbx.get(i, qi);
+                nqr += box_size(A);
+                for (int j = 0; j < nk; ++j) kept += count_kept(m, A, kbx.get(j, c));
+            }
+            cls = rounded_class(kept, nqr * nkr, kpad);
+        } else {
+            bool any = false, all = true;
+            for (int i = 0; i < nq && !(any && !all); ++i) {
+                const Box A = qbx.get(i, qi);
+                for (int j = 0; j < nk; ++j) {
+                    bool ba, bl;
+                    classify_boxes(m, d, sb, A, kbx.get(j, c), ba, bl);
+                    any = any || ba;
+                    all = all && bl;
+                    if (any && !all) break;
+                }
+            }
+            cls = any ? ((all && !kpad) ? VSA_TILE_FULL : VSA_TILE_BOUNDARY) : VSA_TILE_EMPTY;
+        }
+        *out = cls;
+    }
+}
+
 // Per kv tile, one entry per run of bw slots sharing (t, h): the run's t, h,
 // first w and number of real tokens.
 __global__ void seg_table_kernel(vsa_dims d, int2* __restrict__ seg)
@@ -535,6 +645,21 @@ bool tile_fits_unit(int B, int U, int bh, int bw)
 
 unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
 
+// Tiles of at most eight boxes (every frame-0-first tile; tile-major tiles of
+// at most eight units) take the blocked kernel, the rest one thread per cell.
+void launch_tile_map(const vsa_dims& d, const vsa_mask_spec* specs, const uint32_t* sbits, int8_t* map,
+                     cudaStream_t s)
+{
+    const bool few = d.Bq <= kMaxTileBoxes * d.U && d.Bk <= kMaxTileBoxes * d.U && d.heads <= 65535;
+    if (few) {
+        const dim3 g(blocks_for(d.nK, kMapKB), blocks_for(d.nQ, kMapQB), d.heads);
+        tile_map_blocked_kernel<<<g, kMapKB, 0, s>>>(d, specs, sbits, map);
+    } else {
+        const long long cells = (long long)d.heads * d.nQ * d.nK;
+        tile_map_kernel<<<blocks_for(cells, 256), 256, 0, s>>>(d, specs, sbits, map);
+    }
+}
+
 }  // namespace
 
 int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
@@ -549,10 +674,7 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
         stripe_bits_kernel<<<g, 128, 0, s>>>(d, p->d_specs, p->d_sbits);
         VSA_CUDA_TRY(cudaGetLastError());
     }
-    const long long cells = (long long)d.heads * d.nQ * d.nK;
-    tile_map_kernel<<<blocks_for(cells, 256), 256, 0, s>>>(d, p->d_specs,
-                                                          p->has_stripe ? p->d_sbits : nullptr,
-                                                          p->d_map);
+    launch_tile_map(d, p->d_specs, p->has_stripe ? p->d_sbits : nullptr, p->d_map, s);
     VSA_CUDA_TRY(cudaGetLastError());
     kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
         d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
@@ -765,8 +887,7 @@ int vsa_launch_stripe_bits(const vsa_dims& d, const vsa_mask_spec* specs, uint32
 int vsa_launch_tile_map(const vsa_dims& d, const vsa_mask_spec* specs, const uint32_t* sbits, int8_t* map,
                         cudaStream_t s)
 {
-    const long long cells = (long long)d.heads * d.nQ * d.nK;
-    tile_map_kernel<<<blocks_for(cells, 256), 256, 0, s>>>(d, specs, sbits, map);
+    launch_tile_map(d, specs, sbits, map, s);
     return cudaGetLastError() == cudaSuccess ? VSA_OK : VSA_ERR_CUDA;
 }
 

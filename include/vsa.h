@@ -352,7 +352,9 @@ int vsa_ulysses_unpermute(vsa_plan_t plan, const void* o, int B, int D, int rank
  * vsa_permute_qkv + vsa_sparse_attn_fwd + vsa_unpermute; device -> host
  * copies of o and lse.  Two sets of device staging buffers alternate, so
  * chunk c computes while chunk c+1's inputs and chunk c-1's outputs cross
- * PCIe.
+ * PCIe.  Chunks are issued in decreasing order of their plan's executed tile
+ * steps (ties in head order), so the compute left after the last copy in is
+ * the lightest; outputs land at each head's own offset whatever the order.
  *
  * vsa_pipeline_create: same spec / grid / tile arguments and errors as
  * vsa_plan_create, plus B >= 1, D in {64,128}, chunk_heads >= 1; allocates
