@@ -536,10 +536,9 @@ def main():
         return
     world, rank, local = dist_init()
     try:
-        if True:
-            res = run_gpu(args, w, world, rank, local)
-            if rank == 0 and res is not None:
-                print(json.dumps(res), flush=True)
+        res = run_gpu(args, w, world, rank, local)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
     finally:
         if world > 1:
             import torch.distributed as dist
