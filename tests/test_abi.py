@@ -104,6 +104,18 @@ def test_calls_reject_null_plan_on_host():
     h = ctypes.c_void_p()
     assert L.vsa_pipeline_create(None, 1, 2, 2, 2, 1, 1, 1, 128, 128, 1, 128, 1, ctypes.byref(h)) == -1
     assert L.vsa_ulysses_unpermute(None, None, 1, 128, 0, 1, None, None, None) == -1
+    assert L.vsa_plan_kept_pairs(None, None, 0, None) == -1
+    assert L.vsa_tile_map_noalloc(None, 1, 2, 8, 8, 1, 8, 8, 64, 64, None, 0, None) == -1
+    assert L.vsa_plan_create(None, 1, 2, 8, 8, 1, 8, 8, 64, 64, None, ctypes.byref(h)) == -1
+    assert L.vsa_plan_create(None, 1, 2, 8, 8, 1, 8, 8, 64, 64, None, None) == -1
+
+
+def test_every_declared_entry_point_is_checked_here():
+    # each entry point of the header appears in this file's host-side checks
+    # (null arguments above, malformed shapes and strings in the other tests)
+    src = open(__file__).read()
+    for name in sorted(_declared()):
+        assert name in src, name
 
 
 def test_layout_slot_counts():
