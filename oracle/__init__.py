@@ -157,6 +157,24 @@ def attention_rows(spec, grid, unit, D: int, scale: float, q: np.ndarray, k: np.
     return o, lse
 
 
+def attention_dense_real(spec, grid, unit, scale: float, q: np.ndarray, k: np.ndarray,
+                         v: np.ndarray) -> Tuple[np.ndarray, np.ndarray]:
+    """fp64 masked attention of every natural query row from real-valued
+    inputs (any float dtype, e.g. the unrounded fp32 draw), small grids only.
+
+    softmax over the kept keys of scale * q k^T, then times v, with the keep
+    matrix of ``keep_matrix``; the dense formula written out in numpy, so it
+    shares no arithmetic with ``vsa_oracle.c``.  Returns (o [N, D], lse [N]).
+    """
+    q64, k64, v64 = (np.asarray(x, dtype=np.float64) for x in (q, k, v))
+    s = scale * (q64 @ k64.T)
+    s[~keep_matrix(spec, grid, unit)] = -np.inf
+    m = s.max(axis=1, keepdims=True)
+    p = np.exp(s - m)
+    l = p.sum(axis=1, keepdims=True)
+    return (p @ v64) / l, (m + np.log(l))[:, 0]
+
+
 def tile_counts(spec, grid, unit, n_slots: int, Bq: int, Bk: int,
                 qtiles: Optional[Iterable[int]] = None, nthreads: Optional[int] = None
                 ) -> Tuple[np.ndarray, np.ndarray]:

@@ -64,6 +64,33 @@ def test_tiny_all_rows():
     assert counts.tolist() == [[4, 0, 12], [0, 12, 4]]
 
 
+def test_tiny_error_against_the_fp32_draw():
+    """Information: the tiny configuration names fp32 inputs; the kernel sees
+    their bf16 rounding.  Printed per head: the GPU output against the fp64
+    dense attention of the unrounded fp32 draw, next to the share the input
+    rounding alone explains (the oracle on the bf16 values against the same).
+    Asserted only what the parity bound implies by the triangle inequality."""
+    from _helpers import TOL_MAX, TOL_MEAN
+    w = W.tiny()
+    grid = (w.T, w.H, w.W)
+    rows = np.arange(w.N)
+    r = PathRun(w, _inputs(w))
+    try:
+        for h, spec in enumerate(w.specs):
+            draw = [W.head_draw_f32(seed, 0, h, w.N, w.D) for seed in w.seeds]
+            o_f32, _ = oracle.attention_dense_real(spec, grid, w.unit, w.scale, *draw)
+            o_bf16, _ = oracle.attention_rows(spec, grid, w.unit, w.D, w.scale, r.q[0, h], r.k[0, h], r.v[0, h],
+                                              rows)
+            e_gpu = np.abs(r.o_rows(0, h, rows) - o_f32)
+            e_in = np.abs(o_bf16 - o_f32)
+            print(f"tiny head {h}: GPU vs fp32-draw attention max {e_gpu.max():.3e} mean {e_gpu.mean():.3e}; "
+                  f"bf16 input rounding alone max {e_in.max():.3e} mean {e_in.mean():.3e}")
+            assert e_gpu.max() <= e_in.max() + TOL_MAX
+            assert e_gpu.mean() <= e_in.mean() + TOL_MEAN
+    finally:
+        r.close()
+
+
 def test_svg_wan720p():
     w = W.svg_wan720p()
     counts, _ = _check(w, range(w.heads), 96, [0, 7])

@@ -293,6 +293,34 @@ def test_attention_matches_textbook(kind):
         # the full mask is unmasked attention
         o2, _ = _textbook(q, k, v, scale, np.ones((N, N), bool))
         np.testing.assert_allclose(o, o2, rtol=0, atol=1e-12)
+    # the numpy dense form for real-valued inputs agrees with the C oracle on
+    # the same (bf16-valued) numbers
+    o3, lse3 = oracle.attention_dense_real(spec, grid, unit, scale, q, k, v)
+    np.testing.assert_allclose(o3, o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse3, lse, rtol=0, atol=1e-12)
+
+
+def test_attention_dense_real_on_fp32_inputs():
+    """On unrounded fp32 inputs: weights sum to one (v = 1 gives o = 1), lse is
+    the log-sum-exp of the kept scores, and the result moves from the bf16
+    oracle by no more than the input rounding can explain (a few 1e-3)."""
+    g = np.random.default_rng(21)
+    grid, unit, D = (3, 4, 5), (1, 2, 5), 32
+    N = int(np.prod(grid))
+    spec = W.mask_spec("temporal", sink=1, rh=1, rw=1)
+    q, k, v = (g.standard_normal((N, D)).astype(np.float32) for _ in range(3))
+    scale = D ** -0.5
+    keepm = oracle.keep_matrix(spec, grid, unit)
+    o1, lse = oracle.attention_dense_real(spec, grid, unit, scale, q, k, np.ones((N, D), np.float32))
+    np.testing.assert_allclose(o1, 1.0, rtol=0, atol=1e-14)
+    s = scale * (q.astype(np.float64) @ k.astype(np.float64).T)
+    for i in range(N):
+        kept = s[i][keepm[i]]
+        assert abs(lse[i] - (kept.max() + np.log(np.exp(kept - kept.max()).sum()))) < 1e-12
+    o, _ = oracle.attention_dense_real(spec, grid, unit, scale, q, k, v)
+    b16 = [W.bf16_bits_from_f32(x) for x in (q, k, v)]
+    ob, _ = oracle.attention_rows(spec, grid, unit, D, scale, *b16, range(N))
+    assert 0 < np.abs(o - ob).max() < 2e-2
 
 
 def test_attention_weights_sum_to_one():
