@@ -175,6 +175,14 @@ def test_scaling(T, mask):
         assert counts[0].tolist() == [n_tiles - full - bnd, bnd, full]
 
 
+@pytest.mark.parametrize("mask", ["full", "spatial"])
+def test_scaling_T5_all_rows(mask):
+    # the smallest scaling grid (5 x 45 x 80, 18,000 tokens) on every query
+    # row of head 0, each row exact over all keys
+    w = W.scaling(5, mask)
+    _check(w, [0], w.N, [0], qtiles_per_head=4)
+
+
 @pytest.mark.parametrize("q_tile,kv_tile", [(q, k) for q in W.SWEEP_Q for k in W.SWEEP_KV
                                             if (q, k) != (128, 128)])
 def test_tile_sweep(q_tile, kv_tile):
