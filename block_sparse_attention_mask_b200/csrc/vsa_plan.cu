@@ -425,8 +425,8 @@ constexpr int kMapQB = 32;   // q tiles per block
 // (head, 32 q tiles, 128 kv tiles).  Each tile's boxes are derived once per
 // block into shared memory; a thread then classifies its kv tile against the
 // block's 32 q tiles (coalesced byte stores along kv).  Same classes as
-// tile_map_kernel below: any / all kept over the real (A x B) box pairs, or
-// the kept fraction under tile-aligned rounding.
+// tile_map_kernel: any / all kept over the real (A x B) box pairs, or the
+// kept fraction under tile-aligned rounding.
 __global__ void __launch_bounds__(kMapKB) tile_map_blocked_kernel(vsa_dims d,
                                                                   const vsa_mask_spec* __restrict__ specs,
                                                                   const uint32_t* __restrict__ sbits,
