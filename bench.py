@@ -1,6 +1,7 @@
 """Benchmark: block-sparse 3D-video attention on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--partition heads|batch] [--impl reference] [--no-extra]
 
 One step is one pass of the whole path over one batch of synthetic input,
 through the C ABI: rebuild the plan's tile map and kv-tile lists, permute
@@ -19,12 +20,20 @@ q, k, v, the step's kernels and the device-to-host copies of o and lse on
 three streams, overlapped), timed with CUDA events on the caller's stream.
 Routed workloads time it with the copies and the step in series.
 
-N > 1 (torchrun): each rank runs the same workload on its own GPU and its own
-batch element (weak scaling; heads and batches are independent, so there is
-no data-path collective).  Step times are the max over ranks.
+N > 1 (torchrun), --partition heads (default): rank r takes the contiguous
+heads [floor(r H / N), floor((r+1) H / N)) of the same batch element, builds
+its own plan for them and runs the unchanged path (strong scaling: the whole
+job's work is fixed; heads are independent, so there is no data-path
+collective).  --partition batch: every rank runs all heads of its own batch
+element (weak scaling).  Step times are the max over ranks.
 
---impl reference: the CPU oracle (fp64, all host cores) on a bounded sample of
-query rows of the same workload per step, reported in the same unit.
+At N = 1 the line also carries ``workloads``: the attention kernel alone on
+the other workloads (STA HunyuanVideo, the stripe heads, the dense and
+spatial scaling grids T = 5..33 with their scaling efficiency, and the
+q-tile x kv-tile sweep at T = 21), a few timed launches each.
+
+--impl reference: the CPU oracle (fp64, all host cores), each step a bounded
+sample of query rows of the same workload, reported in the same unit.
 """
 from __future__ import annotations
 
@@ -150,10 +159,26 @@ def exec_flops(w, counts) -> float:
 
 
 def rank_workload(w, rank: int):
-    """The workload rank `rank` processes: same shape and masks, its own batch
-    element (independent seeds), so per-GPU work is fixed as ranks are added."""
+    """--partition batch: the workload rank `rank` processes is the same shape
+    and masks with its own batch element (independent seeds), so per-GPU work
+    is fixed as ranks are added."""
     from dataclasses import replace
     return replace(w, seeds=tuple(s + 1000 * rank for s in w.seeds))
+
+
+def head_range(heads: int, rank: int, world: int):
+    """--partition heads: rank r's contiguous heads [floor(r H / G), floor((r+1) H / G))."""
+    if world > heads:
+        raise ValueError(f"{world} ranks for {heads} heads: some rank would hold no head")
+    return rank * heads // world, (rank + 1) * heads // world
+
+
+def rank_shard(w, rank: int, world: int, partition: str):
+    """The workload one rank runs: its head range (heads) or its batch element (batch)."""
+    if partition == "heads":
+        lo, hi = head_range(w.heads, rank, world)
+        return w.head_shard(lo, hi) if (lo, hi) != (0, w.heads) else w
+    return rank_workload(w, rank)
 
 
 def aggregate_tflops(flops_per_rank_step: float, world: int, ms_max: float) -> float:
@@ -183,41 +208,128 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def sum_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
 def barrier(world: int):
     if world > 1:
         import torch.distributed as dist
         dist.barrier()
 
 
-def cpu_baseline(w, seconds_target: float = 12.0):
-    """Time the oracle as it stands on sampled rows of up to four heads with
-    distinct masks and extrapolate linearly (its cost per row does not depend
-    on the row: every row visits all N keys)."""
-    import oracle
-    heads, seen = [], []
+def oracle_groups(w, max_groups: int = 8):
+    """Heads that stand for the workload in an oracle sample: one per distinct
+    mask, with the number of heads sharing it as its weight; with more than
+    ``max_groups`` distinct masks (the stripe workload's 40), ``max_groups``
+    heads spread evenly over the workload, each weighing heads / max_groups."""
+    groups = []
     for h, s in enumerate(w.specs):
-        if s not in seen:
-            seen.append(s)
-            heads.append(h)
-    heads = heads[:4]
+        for g in groups:
+            if w.specs[g[0]] == s:
+                g[1] += 1
+                break
+        else:
+            groups.append([h, 1])
+    if len(groups) > max_groups:
+        pick = np.linspace(0, w.heads - 1, max_groups).round().astype(int)
+        groups = [[int(h), w.heads / max_groups] for h in pick]
+    return [(h, float(c)) for h, c in groups]
+
+
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample_step(w, R: int, seed: int, threads: int):
+    """One bounded sample of the oracle on workload ``w``, timed on host cores.
+
+    For each head standing for the workload (``oracle_groups``): one call with
+    no query rows, which costs what every call costs once (widening the head's
+    k and v to fp64, starting the threads), and one call with R uniform random
+    query rows (each exact over all N keys; a row's cost depends on how many
+    keys its mask keeps, so rows are drawn uniformly, not stratified).
+    Returns (estimated seconds of the oracle over the whole workload: every
+    head pays the fixed cost once and N rows at its mask's per-row cost;
+    wall seconds of this sample; rows timed)."""
+    import oracle
     grid = (w.T, w.H, w.W)
-    threads = oracle.default_threads()
-    spent_all, rows_all = 0.0, 0
-    budget = seconds_target / len(heads)
-    for h in heads:
-        q, k, v = (W.head_tensor(w, x, 0, h) for x in "qkv")
-        R, spent = 64, 0.0
-        while spent < budget and R <= w.N:
-            rows = W.sample_rows(w, h, R, seed=1000 + R)
-            t0 = time.perf_counter()
-            oracle.attention_rows(w.specs[h], grid, w.unit, w.D, w.scale, q, k, v, rows, threads)
-            spent += time.perf_counter() - t0
-            rows_all += len(rows)
-            R *= 2
-        spent_all += spent
-    per_row = spent_all / rows_all
-    est = per_row * w.N * w.heads * w.B
-    return est, threads, spent_all, rows_all, heads
+    est, wall, nrows = 0.0, 0.0, 0
+    for h, weight in oracle_groups(w):
+        key = (w.name, w.head_offset, h)
+        if key not in _ORACLE_INPUTS:
+            if len(_ORACLE_INPUTS) >= 8:
+                _ORACLE_INPUTS.clear()
+            _ORACLE_INPUTS[key] = tuple(W.head_tensor(w, x, 0, h) for x in "qkv")
+        q, k, v = _ORACLE_INPUTS[key]
+        g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, h])))
+        rows = np.sort(g.choice(w.N, size=min(R, w.N), replace=False)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attention_rows(w.specs[h], grid, w.unit, w.D, w.scale, q, k, v, rows[:0], threads)
+        t1 = time.perf_counter()
+        oracle.attention_rows(w.specs[h], grid, w.unit, w.D, w.scale, q, k, v, rows, threads)
+        t2 = time.perf_counter()
+        fixed = t1 - t0
+        per_row = max(0.0, (t2 - t1) - fixed) / len(rows)
+        est += weight * w.B * (fixed + w.N * per_row)
+        wall += t2 - t0
+        nrows += len(rows)
+    return est, wall, nrows
+
+
+def oracle_rate(w, flops_step: float, steps: int, R: int, threads: int, seed0: int = 0):
+    """The oracle's throughput in the bench's unit from ``steps`` samples:
+    executed-tile FLOPs of one whole step over the mean estimated time of the
+    oracle on it.  Both the GPU arm's cpu_baseline and --impl reference call
+    this, so they measure the same thing the same way."""
+    ests, walls, rows = [], [], 0
+    for i in range(steps):
+        e, wl, n = oracle_sample_step(w, R, seed0 + i, threads)
+        ests.append(e)
+        walls.append(wl)
+        rows += n
+    est = statistics.mean(ests)
+    groups = oracle_groups(w)
+    sample = (f"per step, for heads {[h for h, _ in groups]} (weights {[c for _, c in groups]}; one head per "
+              f"distinct mask, or spread evenly): a call with no rows (the per-call fixed cost: widening k, v "
+              f"to fp64, thread start) and a call with {R} uniform random query rows exact over all {w.N} keys; "
+              f"whole-step time estimated as every head's fixed cost + {w.N} rows at its mask's per-row cost "
+              f"= {est:.1f} s (mean of {steps} samples, {rows} rows timed in all)")
+    return flops_step / est / 1e12, est, statistics.mean(walls), sample
+
+
+def oracle_exec_flops(w, threads: int, n_qtiles: int = 64) -> float:
+    """Executed-tile FLOPs of one step of ``w`` from the oracle's own tile
+    classes on ``n_qtiles`` evenly spaced q-tile rows per distinct mask."""
+    import oracle
+    grid = (w.T, w.H, w.W)
+    L = max(128, w.q_tile, w.kv_tile)        # the tile-major slots: padded grid in whole tiles
+    n_slots = -(-oracle.padded_tokens(grid, w.unit) // L) * L
+    nq = n_slots // w.q_tile
+    sample_q = np.unique(np.linspace(0, nq - 1, n_qtiles).round().astype(np.int64))
+    counts, done = np.zeros((w.heads, 3)), {}
+    for h in range(w.heads):
+        key = tuple(sorted(w.specs[h].items()))
+        if key not in done:
+            fn = oracle.rounded_tile_map if w.specs[h].get("tile_round", 0) else oracle.tile_map
+            cls = fn(w.specs[h], grid, w.unit, n_slots, w.q_tile, w.kv_tile, sample_q, threads)
+            done[key] = [(cls == c).sum() * nq / len(sample_q) for c in range(3)]
+        counts[h] = done[key]
+    return exec_flops(w, counts) * w.B
+
+
+def bench_config(w, world: int, partition: str):
+    par = (f"heads{world} (contiguous head ranges per rank, no collective)" if partition == "heads"
+           else f"dp{world} (independent batch per rank)")
+    mb = 3 * w.B * w.heads * w.N * w.D * 2 / 1e6
+    l2 = (f"inputs larger than L2 (natural q,k,v = {mb:.0f} MB), no flush" if mb > 126
+          else f"inputs fit in L2 (natural q,k,v = {mb:.1f} MB): warm-cache timing")
+    return dict(w.describe(), parallelism=par, l2=l2)
 
 
 def run_reference(args, w, world, rank):
@@ -225,53 +337,110 @@ def run_reference(args, w, world, rank):
     if rank != 0:
         return
     import oracle
-    grid = (w.T, w.H, w.W)
     threads = oracle.default_threads()
-    # the tile-major layout holds the padded grid rounded up to whole tiles
-    L = max(128, w.q_tile, w.kv_tile)
-    n_slots = -(-oracle.padded_tokens(grid, w.unit) // L) * L
-    # executed tiles of the workload, from the oracle's own tile classes on sampled q tiles
-    counts = np.zeros((w.heads, 3))
-    nq = n_slots // w.q_tile
-    sample_q = np.unique(np.linspace(0, nq - 1, 8).astype(np.int64))
-    for h in range(w.heads):
-        same = [g for g in range(h) if w.specs[g] == w.specs[h]]
-        if same:
-            counts[h] = counts[same[0]]
-            continue
-        cls = oracle.tile_map(w.specs[h], grid, w.unit, n_slots, w.q_tile, w.kv_tile,
-                              sample_q, threads)
-        for c in range(3):
-            counts[h, c] = (cls == c).sum() * nq / len(sample_q)
-    flops = exec_flops(w, counts) * w.B
-    h0 = 0
-    q, k, v = (W.head_tensor(w, x, 0, h0) for x in "qkv")
+    flops = oracle_exec_flops(w, threads)
     R = 256
-    times = []
-    for step in range(args.warmup + args.steps):
-        rows = W.sample_rows(w, h0, R, seed=step)
-        t0 = time.perf_counter()
-        oracle.attention_rows(w.specs[h0], grid, w.unit, w.D, w.scale, q, k, v, rows, threads)
-        dt = time.perf_counter() - t0
-        if step >= args.warmup:
-            times.append(dt)
-    per_row = statistics.mean(times) / R
-    full_time = per_row * w.N * w.heads * w.B
-    value = flops / full_time / 1e12
-    sample = (f"{R} sampled query rows of head {h0} per step (exact over all {w.N} keys), "
-              f"extrapolated linearly to {w.heads} heads x {w.N} rows; executed tiles from the "
-              f"oracle's classes on {len(sample_q)} sampled q-tile rows per distinct head")
+    for i in range(args.warmup):              # untimed: page in inputs, warm the caches
+        oracle_sample_step(w, 16, 10_000 + i, threads)
+    value, est, wall, sample = oracle_rate(w, flops, args.steps, R, threads)
+    sample += (f"; executed tiles from the oracle's classes on 64 evenly spaced q-tile rows per distinct mask; "
+               f"ms_per_step is the wall time of one sample step")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": full_time * 1e3, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": wall * 1e3, "higher_is_better": True,
+        "scaling": "strong" if args.partition == "heads" else "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": dict(w.describe(), parallelism="cpu oracle"),
+        "config": bench_config(w, args.gpus, args.partition),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "est_step_s": est},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+EXTRA_WARMUP, EXTRA_TIMED = 3, 5
+
+
+def extra_entries():
+    """(key, workload) pairs timed for the line's ``workloads`` key."""
+    out = [("sta_hunyuan720p", W.sta_hunyuan720p()), ("stripe_wan720p", W.stripe_wan720p())]
+    for T in W.SCALING_T:
+        for m in ("full", "spatial"):
+            out.append((f"scaling_{m}_T{T}", W.scaling(T, m)))
+    for q in W.SWEEP_Q:
+        for k in W.SWEEP_KV:
+            if (q, k) != (128, 128):
+                out.append((f"sweep_q{q}_k{k}", W.scaling(21, "spatial", q, k)))
+    return out
+
+
+def time_attention(w, dev, stream, peak: float) -> dict:
+    """The attention kernel alone on workload ``w``: plan, permuted N(0,1)
+    bf16 inputs drawn on the device from a fixed seed, EXTRA_WARMUP untimed and
+    EXTRA_TIMED timed launches (CUDA events on the launching stream)."""
+    import torch
+    import block_sparse_attention_mask_b200 as vsa
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(1234)
+    with torch.cuda.stream(stream):
+        plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile, stream=stream)
+        try:
+            S = plan.n_slots
+            nat = [torch.randn((w.B, w.heads, w.N, w.D), generator=gen, device=dev).to(torch.bfloat16)
+                   for _ in range(3)]
+            qp = torch.empty((w.B, w.heads, S, w.D), dtype=torch.bfloat16, device=dev)
+            kp, vp, op = torch.empty_like(qp), torch.empty_like(qp), torch.empty_like(qp)
+            lse = torch.empty((w.B, w.heads, S), dtype=torch.float32, device=dev)
+            h, sh = plan.handle, stream.cuda_stream
+            vsa.vsa_permute_qkv(h, nat[0], nat[1], nat[2], qp, kp, vp, w.B, w.D, sh)
+            del nat
+            for _ in range(EXTRA_WARMUP):
+                vsa.vsa_sparse_attn_fwd(qp, kp, vp, op, lse, h, w.B, w.D, w.scale, sh)
+            ev = []
+            for _ in range(EXTRA_TIMED):
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                vsa.vsa_sparse_attn_fwd(qp, kp, vp, op, lse, h, w.B, w.D, w.scale, sh)
+                e1.record(stream)
+                ev.append((e0, e1))
+            stream.synchronize()
+            plan.check(stream)
+            counts = plan.tile_counts(stream)
+            steps = int(plan.exec_steps(stream).sum())
+        finally:
+            plan.close()
+    ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = exec_flops(w, counts) * w.B
+    tf = flops / (ms * 1e-3) / 1e12
+    full, bnd, empty = (int(counts[:, c].sum()) for c in (2, 1, 0))
+    return {"fwd_ms": round(ms, 4), "tflops": round(tf, 1), "frac": round(tf / peak, 4),
+            "exec_tflop": round(flops / 1e12, 4), "tiles": {"full": full, "boundary": bnd, "empty": empty},
+            "boundary_share": round(bnd / max(1, full + bnd), 4),
+            "executed_fraction": round((full + bnd) / max(1, full + bnd + empty), 4), "exec_steps": steps,
+            "q_tile": w.q_tile, "kv_tile": w.kv_tile}
+
+
+def extra_workloads(dev, stream, peak: float, smi_id: str) -> dict:
+    """Attention-only numbers for the other workloads, and the scaling
+    efficiency (t_spatial / t_dense) / (executed spatial / executed dense)
+    per T: 1 means the wall time follows the executed-tile fraction."""
+    smi = ClockSampler(smi_id)
+    smi.start()
+    out = {}
+    for key, w in extra_entries():
+        out[key] = time_attention(w, dev, stream, peak)
+    clk = smi.stop()
+    eff = {}
+    for T in W.SCALING_T:
+        d, sp = out[f"scaling_full_T{T}"], out[f"scaling_spatial_T{T}"]
+        eff[f"T{T}"] = round((sp["fwd_ms"] / d["fwd_ms"]) / (sp["exec_tflop"] / d["exec_tflop"]), 4)
+    out["scaling_efficiency"] = eff
+    out["timing"] = (f"attention kernel alone, {EXTRA_TIMED} launches after {EXTRA_WARMUP} warm-ups, CUDA events; "
+                     f"frac of the measured burst bf16 peak {peak}")
+    out["clocks"] = clk
+    return out
 
 
 def run_gpu(args, w, world, rank, local):
@@ -284,9 +453,10 @@ def run_gpu(args, w, world, rank, local):
     grid = (w.T, w.H, w.W)
     B = w.B
 
-    # inputs: rank r draws its own batch element (weak scaling)
-    wr = rank_workload(w, rank)
-    host = [W.full_tensor(wr, x) for x in "qkv"]
+    # this rank's share: its head range (default) or its own batch element
+    wg = w
+    w = rank_shard(w, rank, world, args.partition)
+    host = [W.full_tensor(w, x) for x in "qkv"]
     pinned = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in host]
     del host
     with torch.cuda.stream(stream):
@@ -389,7 +559,9 @@ def run_gpu(args, w, world, rank, local):
         if routed else None
     ms_step = max_over_ranks(statistics.mean(ms_steps), world, dev)
     ms_fwd_mean = max_over_ranks(statistics.mean(ms_fwd), world, dev)
-    value = aggregate_tflops(flops_step, world, ms_step)
+    # whole-job executed FLOPs: every rank's own (head ranges differ in work)
+    flops_job = sum_over_ranks(flops_step, world, dev)
+    value = flops_job / (ms_step * 1e-3) / 1e12
 
     # ---- end to end through the public API with host buffers ----
     o_host = torch.empty(o.shape, dtype=torch.bfloat16).pin_memory()
@@ -442,7 +614,8 @@ def run_gpu(args, w, world, rank, local):
 
     pk, how = peaks()
     peak = float(pk.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
-    achieved = flops_b * B / (ms_fwd_mean * 1e-3) / 1e12
+    # the dominant kernel on this rank: its executed FLOPs over its own mean launch time
+    achieved = flops_b * B / (statistics.mean(ms_fwd) * 1e-3) / 1e12
     traffic = None
     prof = os.path.join(ROOT, "profiles", "attn_fwd_svg_wan720p_traffic.txt")
     if os.path.exists(prof):
@@ -454,37 +627,40 @@ def run_gpu(args, w, world, rank, local):
         except Exception:
             traffic = None
 
+    kept = plan.kept_pairs(stream)
+    useful = sum_over_ranks(4.0 * w.D * float(kept.sum()) * B, world, dev)
+    tiles = [sum_over_ranks(float(counts[:, c].sum()), world, dev) for c in range(3)]
+    extra = None
+    if world == 1 and not args.no_extra:
+        extra = extra_workloads(dev, stream, float(peaks()[0].get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+                                smi_id)
     result = None
     if rank == 0:
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            est, cores, spent, nrows, heads = cpu_baseline(w)
-            cpu = {"value": flops_step / est / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                   "sample": (f"{nrows} stratified query rows of heads {heads} (one per distinct mask, "
-                              f"exact over all {w.N} keys, {spent:.1f} s), extrapolated linearly to "
-                              f"{w.heads} heads x {w.N} rows = {est:.0f} s for one step")}
-        kept = plan.kept_pairs(stream)
-        useful = 4.0 * w.D * float(kept.sum()) * B
+            import oracle
+            threads = oracle.default_threads()
+            cval, est, _, sample = oracle_rate(w, flops_step, 4, 512, threads, seed0=100)
+            cpu = {"value": cval, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                   "sample": sample, "est_step_s": est}
+        heads_job = wg.heads if args.partition == "heads" else wg.heads * world
         result = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic",
-            "config": dict(w.describe(), parallelism=f"dp{world} (independent batch per rank)",
-                           l2="inputs larger than L2 (natural q,k,v = "
-                              f"{3 * q.numel() * 2 / 1e6:.0f} MB), no flush"),
+            "higher_is_better": True, "scaling": "strong" if args.partition == "heads" else "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": bench_config(wg, world, args.partition),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "kernel": "attn_fwd_kernel<128,128>",
                          "peak_source": f"{how} bf16_tflops (burst)"},
             "fwd_ms": ms_fwd_mean,
-            "exec_tflop_per_step": flops_step / 1e12,
+            "exec_tflop_per_step": flops_job / 1e12,
             "useful_tflop_per_step": useful / 1e12,
             "useful_tflops_fwd": useful / (ms_fwd_mean * 1e-3) / 1e12,
-            "kept_pair_fraction": float(kept.sum()) / (w.heads * w.N ** 2),
-            "tiles": {"full": int(counts[:, 2].sum()), "boundary": int(counts[:, 1].sum()),
-                      "empty": int(counts[:, 0].sum()),
-                      "boundary_share_of_executed": float(counts[:, 1].sum() / max(1, counts[:, 1:].sum()))},
+            "kept_pair_fraction": useful / (4.0 * w.D * B) / (heads_job * w.N ** 2),
+            "tiles": {"full": int(tiles[2]), "boundary": int(tiles[1]), "empty": int(tiles[0]),
+                      "boundary_share_of_executed": tiles[1] / max(1.0, tiles[1] + tiles[2])},
             "exec_steps": int(steps_exec.sum()),
             "cpu_baseline": cpu,
             "route": None if not routed else {
@@ -493,11 +669,14 @@ def run_gpu(args, w, world, rank, local):
                 # four R x N x D products (QK^T and three PV) over the sampled rows
                 "tflops": 8.0 * B * w.heads * len(rows_np) * w.N * w.D / (ms_route * 1e-3) / 1e12,
                 "frac": 8.0 * B * w.heads * len(rows_np) * w.N * w.D / (ms_route * 1e-3) / 1e12 / peak},
-            "e2e": {"value": aggregate_tflops(flops_step, world, ms_e2e), "unit": "TFLOP/s",
-                    "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "e2e": {"value": flops_job / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+                    "ms_per_step": ms_e2e, "h2d_bytes_per_step": h2d * world,
+                    "d2h_bytes_per_step": d2h * world},
             "clocks": clk,
-            "gpu_launches": per_step_launches * args.steps,
+            "gpu_launches": per_step_launches * args.steps * world,
         }
+        if extra is not None:
+            result["workloads"] = extra
     plan.close()
     return result
 
@@ -526,6 +705,9 @@ def main():
     ap.add_argument("--workload", default="svg_wan720p", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="vsa", choices=["vsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the other workloads' attention timings")
+    ap.add_argument("--partition", default="heads", choices=["heads", "batch"],
+                    help="N > 1: split the heads across ranks (default) or give each rank a batch element")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

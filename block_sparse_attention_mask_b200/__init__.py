@@ -247,11 +247,22 @@ def vsa_sparse_attn_fwd(q, k, v, o, lse, plan: int, B: int, D: int, scale: float
 
 def vsa_tile_map_noalloc(specs: Sequence[Dict[str, int]], grid: Sequence[int], unit: Sequence[int],
                          q_tile: int, kv_tile: int, map_out, stream=None) -> None:
-    """Tile map into a caller-owned int8 CUDA tensor; the library allocates nothing."""
+    """Tile map into a caller-owned int8 CUDA tensor; the library allocates nothing.
+
+    ``map_out`` must be a contiguous int8 CUDA tensor on the current device;
+    the bound passed to the library is the bytes its storage really holds from
+    the tensor's first element on, so a view can never let the kernel write
+    past its allocation."""
+    import torch
+    if not (isinstance(map_out, torch.Tensor) and map_out.is_cuda and map_out.dtype == torch.int8
+            and map_out.is_contiguous() and map_out.device.index == torch.cuda.current_device()):
+        raise VsaError(-1, "vsa_tile_map_noalloc: map_out must be a contiguous int8 CUDA tensor "
+                           "on the current device")
     arr = (vsa_mask_spec * len(specs))(*[make_spec(s) for s in specs])
     T, H, W = (int(x) for x in grid)
     bt, bh, bw = (int(x) for x in unit)
-    nbytes = map_out.numel() * map_out.element_size() if hasattr(map_out, "numel") else 0
+    nbytes = min(map_out.numel(),
+                 map_out.untyped_storage().nbytes() - map_out.storage_offset() * map_out.element_size())
     _check(_lib.vsa_tile_map_noalloc(arr, len(specs), T, H, W, bt, bh, bw, int(q_tile), int(kv_tile),
                                      _ptr(map_out), nbytes, _stream(stream)),
            "vsa_tile_map_noalloc")

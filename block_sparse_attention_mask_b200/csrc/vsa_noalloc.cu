@@ -85,6 +85,21 @@ extern "C" int vsa_tile_map_noalloc(const vsa_mask_spec* specs, int num_heads, i
     const size_t need_scratch = kSpecBytes + (size_t)num_heads * d.sbits_words * sizeof(uint32_t);
     if (need_scratch > VSA_NOALLOC_SCRATCH_BYTES) return VSA_ERR_UNSUPPORTED;
 
+    // map_out must be device (or managed) memory of the current device: a host
+    // pointer or another GPU's memory would fault the kernel, so it is refused
+    // here (cudaPointerGetAttributes allocates nothing)
+    {
+        int dev = -1;
+        if (cudaGetDevice(&dev) != cudaSuccess) return VSA_ERR_CUDA;
+        cudaPointerAttributes pa;
+        memset(&pa, 0, sizeof pa);
+        if (cudaPointerGetAttributes(&pa, map_out) != cudaSuccess) {
+            cudaGetLastError();
+            return VSA_ERR_INVALID_ARG;
+        }
+        if ((pa.type != cudaMemoryTypeDevice && pa.type != cudaMemoryTypeManaged) || pa.device != dev)
+            return VSA_ERR_INVALID_ARG;
+    }
     void* base = nullptr;
     {
         const int r = scratch_address(&base);

@@ -209,7 +209,11 @@ int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stre
  * Writes the same int8 map [num_heads][n_q_tiles][n_kv_tiles] that
  * vsa_plan_create builds (arguments and supported shapes as there) into
  * `map_out`, caller-owned device memory of `map_bytes` >= the map size
- * (vsa_layout_info gives it).  Asynchronous on `stream`.
+ * (vsa_layout_info gives it).  Asynchronous on `stream`.  `map_out` must be
+ * device or managed memory of the current device (checked with
+ * cudaPointerGetAttributes, which allocates nothing; VSA_ERR_INVALID_ARG
+ * otherwise), and `map_bytes` must not exceed what the caller really owns
+ * from `map_out` on: the kernel writes the whole map.
  *
  * Working memory is one file-scope device array of VSA_NOALLOC_SCRATCH_BYTES
  * that every GPU loading the library holds until the process exits; it keeps
@@ -219,7 +223,10 @@ int vsa_plan_kept_pairs(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stre
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  * The first call on a device looks up the array's device address with
  * cudaGetSymbolAddress (once per device, with that device current); make that
- * first call before any stream capture.  All calls share the array and it
+ * first call before any stream capture.  The address is cached for the life
+ * of the process: after cudaDeviceReset (or anything else that destroys the
+ * device's primary context) it is stale, so do not call this entry point on
+ * that device again in the same process.  All calls share the array and it
  * keeps the last call's contents (each call rewrites what it reads), so calls
  * that overlap on the GPU race: serialise them, e.g. on one stream. */
 #define VSA_NOALLOC_SCRATCH_BYTES (1u << 20)

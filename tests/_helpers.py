@@ -102,6 +102,58 @@ def oracle_map_rows(w: W.Workload, h: int, n_slots: int, qtiles) -> np.ndarray:
     return fn(w.specs[h], (w.T, w.H, w.W), w.unit, n_slots, w.q_tile, w.kv_tile, qtiles)
 
 
+_FULL_MAPS = None
+
+
+def full_maps() -> dict:
+    """The oracle's full-size map digests, tile counts and q-tile strata per
+    parity workload (``tests/golden/full_maps.json``)."""
+    global _FULL_MAPS
+    if _FULL_MAPS is None:
+        import json
+        import os
+        path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "full_maps.json")
+        with open(path) as f:
+            _FULL_MAPS = json.load(f)["workloads"]
+    return _FULL_MAPS
+
+
+def heads_of(rec: dict) -> list:
+    """Per-head view of a workload record of ``full_maps()``: each head's mask record."""
+    return [rec["maps"][i] for i in rec["head_mask"]]
+
+
+def parity_rows(w: W.Workload, h: int, R: int = 512, seed: int = 7) -> np.ndarray:
+    """R stratified natural query rows of head h for a sampled parity check.
+
+    The strata of ``workloads.sample_rows`` (frame 0, the last frame, the
+    padded-edge latent rows, the grid corners, uniform rows) plus rows of q
+    tiles whose executed kv tiles are all boundary and of q tiles whose
+    executed kv tiles are all full, as the oracle's full map of the head
+    classifies them (q tiles listed in ``tests/golden/full_maps.json``).  Up
+    to R/4 rows come from those q tiles, spread evenly over them."""
+    rec = full_maps()[w.name]
+    head = heads_of(rec)[h]
+    perm = oracle.tile_major_order((w.T, w.H, w.W), w.unit, rec["n_slots"],
+                                   layout=int(w.specs[h].get("layout", 0)))
+    tiles = head["boundary_only_qtiles"] + head["full_only_qtiles"]
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([seed, h, 1])))
+    picks = {}
+    if tiles:
+        per_tile = max(1, (R // 4) // len(tiles))
+        for qt in tiles:
+            nat = perm[qt * w.q_tile:(qt + 1) * w.q_tile]
+            nat = nat[nat >= 0]
+            for n in g.choice(nat, size=min(per_tile, len(nat)), replace=False):
+                picks[int(n)] = None
+    target = min(R, w.N)
+    for n in W.sample_rows(w, h, max(1, target - len(picks)), seed=seed):
+        picks[int(n)] = None
+    while len(picks) < target:                  # rows both strata picked
+        picks[int(g.integers(0, w.N))] = None
+    return np.array(sorted(picks), dtype=np.int64)
+
+
 def sample_qtiles(n_q: int, k: int, seed: int) -> np.ndarray:
     g = np.random.default_rng(seed)
     pick = {0, n_q - 1, n_q // 2}

@@ -1,17 +1,21 @@
 """GPU parity at the full workload sizes, in the launch configuration the
 benchmark times (all heads, B = 1, the workload's tile shape).
 
-Outputs are compared with the oracle on stratified sampled rows (frame 0, last
-frame, the padded edge, corners, random), each row exact over all N keys.
-Tile maps are compared with the oracle's brute-force classes on sampled q-tile
-rows, and their per-head totals with closed forms where one exists.
+Outputs are compared with the oracle on R = 512 stratified sampled rows per
+head (frame 0, last frame, the padded edge, corners, rows of q tiles whose
+executed kv tiles are all boundary or all full, uniform rows), each row exact
+over all N keys, on every head of the SVG, STA and stripe workloads and on
+the first and last head of each scaling grid (both of its masks).  Tile maps
+are compared with the oracle's brute-force classes on sampled q-tile rows
+here, and bit for bit on every head in ``test_gpu_full_maps.py``; their
+per-head totals also with closed forms where one exists.
 """
 import numpy as np
 import pytest
 
 import oracle
 import workloads as W
-from _helpers import PathRun, oracle_map_rows, sample_qtiles
+from _helpers import PathRun, oracle_map_rows, parity_rows, sample_qtiles
 
 pytestmark = pytest.mark.gpu
 
@@ -31,7 +35,8 @@ def _check(w, heads, rows_per_head, map_heads, qtiles_per_head=6):
     try:
         errs = []
         for h in heads:
-            errs.append(r.check_rows(h, W.sample_rows(w, h, rows_per_head)))
+            rows = np.arange(w.N) if rows_per_head >= w.N else parity_rows(w, h, rows_per_head)
+            errs.append(r.check_rows(h, rows))
         gmap = r.plan.tile_map()
         for h in map_heads:
             qt = sample_qtiles(gmap.shape[1], qtiles_per_head, seed=h)
@@ -93,7 +98,7 @@ def test_tiny_error_against_the_fp32_draw():
 
 def test_svg_wan720p():
     w = W.svg_wan720p()
-    counts, _ = _check(w, range(w.heads), 96, [0, 7])
+    counts, _ = _check(w, range(w.heads), 512, [0, 7])
     for h in range(5):
         assert counts[h].tolist() == [324900, 12000, 60000]
     for h in range(5, 10):
@@ -111,7 +116,7 @@ def test_svg_wan720p_temporal_frame0_first():
     # sampled q tiles against the oracle in that order, outputs of sampled
     # rows, and the layout-invariant kept pairs; far fewer executed tiles
     w = W.svg_wan720p(temporal_layout=1)
-    counts, _ = _check(w, [0, 5, 9], 96, [5, 9], qtiles_per_head=8)
+    counts, _ = _check(w, range(w.heads), 512, [5, 9], qtiles_per_head=8)
     for h in range(5):
         assert counts[h].tolist() == [324900, 12000, 60000]
     base = W.svg_wan720p()
@@ -134,7 +139,7 @@ def test_svg_wan720p_tile_rounded(layout):
     # against the oracle's rounded map, sampled rows against attention under
     # the rounded mask; boundary tiles remain only where a kv tile has padding
     w = W.svg_wan720p(temporal_layout=layout, tile_round=1)
-    counts, _ = _check(w, [0, 5, 9], 64, [0, 5], qtiles_per_head=6)
+    counts, _ = _check(w, [0, 5, 9], 512, [0, 5], qtiles_per_head=6)
     import block_sparse_attention_mask_b200 as vsa
     plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile)
     try:
@@ -149,7 +154,7 @@ def test_svg_wan720p_tile_rounded(layout):
 
 def test_sta_hunyuan720p():
     w = W.sta_hunyuan720p()
-    counts, _ = _check(w, [0, 11, 23], 96, [0])
+    counts, _ = _check(w, range(w.heads), 512, [0])
     # 900 q tiles of 128 each see 45 window units x 3 tiles; no boundary tiles
     for h in range(w.heads):
         assert counts[h].tolist() == [810000 - 121500, 0, 121500]
@@ -157,7 +162,7 @@ def test_sta_hunyuan720p():
 
 def test_stripe_wan720p():
     w = W.stripe_wan720p()
-    counts, _ = _check(w, range(w.heads), 20, range(0, 40, 3), qtiles_per_head=4)
+    counts, _ = _check(w, range(w.heads), 512, range(0, 40, 3), qtiles_per_head=4)
     assert (counts.sum(axis=1) == 630 * 630).all()
 
 
@@ -165,7 +170,7 @@ def test_stripe_wan720p():
 @pytest.mark.parametrize("mask", ["full", "spatial"])
 def test_scaling(T, mask):
     w = W.scaling(T, mask)
-    counts, _ = _check(w, [0, 39], 48, [0])
+    counts, _ = _check(w, [0, 39], 512, [0])
     n_tiles = (3840 * T // 128) ** 2
     if mask == "full":
         # only the kv tiles holding padded rows (5 of 30 per frame) are boundary
@@ -187,7 +192,7 @@ def test_scaling_T5_all_rows(mask):
                                             if (q, k) != (128, 128)])
 def test_tile_sweep(q_tile, kv_tile):
     w = W.scaling(21, "spatial", q_tile, kv_tile)
-    counts, _ = _check(w, [0, 39], 48, [0])
+    counts, _ = _check(w, [0, 39], 512, [0])
     full, bnd = _spatial_closed_form(21, q_tile, kv_tile)
     assert counts[0][2] == full and counts[0][1] == bnd
     assert bnd * 5 == full  # boundary share of executed tiles is 1/6

@@ -5,7 +5,12 @@ themselves (a framework-owned memory pool, or a serving loop that cannot
 afford cudaMalloc's device synchronisation).  It keeps its working memory in
 one static device array shared by every call, so these tests call it through
 the C ABI several times in a row, with different head counts and grid sizes,
-and require each map to equal, bit for bit, the map vsa_plan_create builds.
+and require each map to equal, bit for bit, the map vsa_plan_create builds,
+and the device's free memory to stay the same across the calls.
+
+Every pointer handed to the C entry point here is a real buffer of the size
+the call is told: a rejection test never relies on the order of the host-side
+checks to keep a kernel from running.
 """
 import ctypes
 
@@ -16,21 +21,28 @@ import block_sparse_attention_mask_b200 as vsa
 import workloads as W
 
 S = W.mask_spec
+MAX_HEADS = 64
 
 
-def _noalloc(specs, grid, unit, q_tile, kv_tile):
-    import torch
-    info = vsa.vsa_layout_info(len(specs), grid, unit, q_tile, kv_tile)
-    out = torch.full((info["map_bytes"],), -1, dtype=torch.int8, device="cuda")
+def _raw_call(specs, grid, unit, q_tile, kv_tile, ptr, nbytes, stream):
     arr = (vsa.vsa_mask_spec * len(specs))(*[vsa.make_spec(s) for s in specs])
     T, H, Wd = grid
     bt, bh, bw = unit
-    rc = vsa.lib.vsa_tile_map_noalloc(arr, len(specs), T, H, Wd, bt, bh, bw, q_tile, kv_tile,
-                                      ctypes.c_void_p(out.data_ptr()), out.numel(),
-                                      ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    return vsa.lib.vsa_tile_map_noalloc(arr, len(specs), T, H, Wd, bt, bh, bw, q_tile, kv_tile,
+                                        ctypes.c_void_p(ptr), nbytes, ctypes.c_void_p(stream))
+
+
+def _out_buffer(specs, grid, unit, q_tile, kv_tile):
+    import torch
+    info = vsa.vsa_layout_info(len(specs), grid, unit, q_tile, kv_tile)
+    out = torch.full((info["map_bytes"],), -1, dtype=torch.int8, device="cuda")
+    return out, (len(specs), info["n_q_tiles"], info["n_kv_tiles"])
+
+
+def _noalloc_into(out, call):
+    import torch
+    rc = _raw_call(*call, out.data_ptr(), out.numel(), torch.cuda.current_stream().cuda_stream)
     assert rc == 0, vsa.vsa_status_string(rc)
-    torch.cuda.synchronize()
-    return out.cpu().numpy().reshape(len(specs), info["n_q_tiles"], info["n_kv_tiles"])
 
 
 def _with_plan(specs, grid, unit, q_tile, kv_tile):
@@ -56,25 +68,80 @@ CALLS = [
 
 @pytest.mark.gpu
 def test_noalloc_map_equals_plan_map_on_consecutive_calls():
-    got = [_noalloc(*c) for c in CALLS]          # back to back, sharing the scratch
+    import torch
+    outs = [_out_buffer(*c) for c in CALLS]
+    # one call of each kind first: the first launch of a kernel may load its
+    # module, which is the library's one-time set-up, not the call's
+    for c, (o, _) in zip(CALLS, outs):
+        _noalloc_into(o, c)
+    again = torch.full_like(outs[1][0], -1)
+    for o, _ in outs:
+        o.fill_(-1)
+    torch.cuda.synchronize()
+    free0, _ = torch.cuda.mem_get_info()
+    alloc0 = torch.cuda.memory_allocated()
+    for c, (o, _) in zip(CALLS, outs):         # back to back, sharing the scratch
+        _noalloc_into(o, c)
+    _noalloc_into(again, CALLS[1])             # a repeat after a different call
+    torch.cuda.synchronize()
+    free1, _ = torch.cuda.mem_get_info()
+    # neither torch's allocator nor the device saw an allocation
+    assert torch.cuda.memory_allocated() == alloc0
+    assert free1 == free0, f"device free memory changed by {free0 - free1} bytes"
+    got = [o.cpu().numpy().reshape(shape) for o, shape in outs]
     for c, g in zip(CALLS, got):
         assert (g == _with_plan(*c)).all()
-    again = _noalloc(*CALLS[1])                  # a repeat after a different call
-    assert (again == got[1]).all()
+    assert (again.cpu().numpy().reshape(outs[1][1]) == got[1]).all()
 
 
+@pytest.mark.gpu
 def test_noalloc_rejects_requests_beyond_its_scratch():
-    spec = vsa.make_spec(S("stripe", 0, Tw=1, To=0, Ts=2, Sw=1, So=0, Ss=3))
-    many = (vsa.vsa_mask_spec * (vsa_max_heads() + 1))(*([spec] * (vsa_max_heads() + 1)))
-    rc = vsa.lib.vsa_tile_map_noalloc(many, vsa_max_heads() + 1, 4, 8, 8, 1, 8, 8, 64, 64,
-                                      ctypes.c_void_p(16), 1 << 20, None)
-    assert rc == -2
+    import torch
+    spec = S("stripe", 0, Tw=1, To=0, Ts=2, Sw=1, So=0, Ss=3)
+    stream = torch.cuda.current_stream().cuda_stream
+    # more heads than the spec area holds
+    call = ([spec] * (MAX_HEADS + 1), (4, 8, 8), (1, 8, 8), 64, 64)
+    out, _ = _out_buffer(*call)
+    assert _raw_call(*call, out.data_ptr(), out.numel(), stream) == -2
     # 64 stripe heads on a 256 x 256 frame need about 2 MiB of offset tables
-    big = (vsa.vsa_mask_spec * 64)(*([spec] * 64))
-    rc = vsa.lib.vsa_tile_map_noalloc(big, 64, 1, 256, 256, 1, 8, 8, 64, 64,
-                                      ctypes.c_void_p(16), 1 << 30, None)
-    assert rc == -2
+    call = ([spec] * MAX_HEADS, (1, 256, 256), (1, 8, 8), 64, 64)
+    out, _ = _out_buffer(*call)
+    assert _raw_call(*call, out.data_ptr(), out.numel(), stream) == -2
+    torch.cuda.synchronize()
+    assert (out == -1).all()                   # nothing was written
 
 
-def vsa_max_heads():
-    return 64
+@pytest.mark.gpu
+def test_noalloc_rejects_a_map_that_is_not_device_memory():
+    import torch
+    call = CALLS[1]
+    out, _ = _out_buffer(*call)
+    host = torch.full((out.numel(),), -1, dtype=torch.int8).pin_memory()
+    stream = torch.cuda.current_stream().cuda_stream
+    assert _raw_call(*call, host.data_ptr(), host.numel(), stream) == -1
+    # a map buffer smaller than the map
+    assert _raw_call(*call, out.data_ptr(), out.numel() - 1, stream) == -1
+    torch.cuda.synchronize()
+    assert (host == -1).all() and (out == -1).all()
+    # the Python wrapper refuses views and wrong types before the C call
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_tile_map_noalloc(call[0], *call[1:], out[::2])
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_tile_map_noalloc(call[0], *call[1:], host)
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_tile_map_noalloc(call[0], *call[1:], out.view(torch.uint8))
+    # a view that starts inside a buffer is bounded by what remains of it
+    with pytest.raises(vsa.VsaError):
+        vsa.vsa_tile_map_noalloc(call[0], *call[1:], out[1:])
+    vsa.vsa_tile_map_noalloc(call[0], *call[1:], out)
+    torch.cuda.synchronize()
+    assert (out.cpu().numpy().reshape(_out_buffer(*call)[1]) == _with_plan(*call)).all()
+
+
+def test_noalloc_rejects_bad_arguments_on_the_host():
+    """Null buffers and head counts out of range are refused before any
+    device work; no pointer other than NULL is passed."""
+    spec = S("spatial", 1, rt=1)
+    assert _raw_call([spec], (4, 8, 8), (1, 8, 8), 64, 64, None, 1 << 20, None) == -1
+    arr = (vsa.vsa_mask_spec * 1)(vsa.make_spec(spec))
+    assert vsa.lib.vsa_tile_map_noalloc(arr, 0, 4, 8, 8, 1, 8, 8, 64, 64, None, 1 << 20, None) == -1

@@ -91,6 +91,9 @@ class Workload:
     structure_amp: float = 0.0
     # candidate masks for SVG routing (one pair per head), empty if not routed
     route_specs: Tuple[Tuple[Dict[str, int], Dict[str, int]], ...] = ()
+    # global index of local head 0: a shard holding heads [lo, hi) of a
+    # workload draws exactly the inputs those heads have in the whole one
+    head_offset: int = 0
 
     @property
     def N(self) -> int:
@@ -104,6 +107,16 @@ class Workload:
                    unit: Optional[Tuple[int, int, int]] = None) -> "Workload":
         return replace(self, q_tile=q_tile, kv_tile=kv_tile,
                        unit=unit if unit is not None else self.unit)
+
+    def head_shard(self, lo: int, hi: int) -> "Workload":
+        """Heads [lo, hi) of this workload as a workload of their own (same
+        grid, tiles and per-head masks; inputs drawn as in the whole one)."""
+        if not 0 <= lo < hi <= self.heads:
+            raise ValueError(f"head range [{lo}, {hi}) outside {self.heads} heads")
+        return replace(self, heads=hi - lo, specs=self.specs[lo:hi],
+                       structure=self.structure[lo:hi] if self.structure else (),
+                       route_specs=self.route_specs[lo:hi] if self.route_specs else (),
+                       head_offset=self.head_offset + lo)
 
     def describe(self) -> Dict[str, object]:
         return {"workload": self.name, "B": self.B, "grid": [self.T, self.H, self.W],
@@ -247,6 +260,7 @@ def structure_embedding(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray]:
     of head ``h``: class = frame t for "frame", (h, w) position for
     "position".  Drawn from ``PCG64(SeedSequence([seeds[0] + 1000, h]))``."""
     kind = w.structure[h]
+    hg = w.head_offset + h
     n = np.arange(w.N)
     if kind == "frame":
         cls, C = n // (w.H * w.W), w.T
@@ -254,7 +268,7 @@ def structure_embedding(w: Workload, h: int) -> Tuple[np.ndarray, np.ndarray]:
         cls, C = n % (w.H * w.W), w.H * w.W
     else:
         raise ValueError(f"no structure for head {h}")
-    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seeds[0] + 1000, h])))
+    g = np.random.Generator(np.random.PCG64(np.random.SeedSequence([w.seeds[0] + 1000, hg])))
     e = g.standard_normal((C, w.D))
     e /= np.linalg.norm(e, axis=1, keepdims=True)
     return cls, e.astype(np.float32)
@@ -267,7 +281,7 @@ def head_tensor(w: Workload, which: str, b: int, h: int) -> np.ndarray:
     head's embedding of each token's class added to the N(0,1) draw before
     the bf16 rounding; v stays iid."""
     seed = w.seeds["qkv".index(which)]
-    x = head_draw_f32(seed, b, h, w.N, w.D)
+    x = head_draw_f32(seed, b, w.head_offset + h, w.N, w.D)
     if which in "qk" and w.structure and w.structure[h]:
         cls, e = structure_embedding(w, h)
         x += np.float32(w.structure_amp) * e[cls]
