@@ -303,15 +303,19 @@ def oracle_rate(w, flops_step: float, steps: int, R: int, threads: int, seed0: i
     return flops_step / est / 1e12, est, statistics.mean(walls), sample
 
 
-def oracle_exec_flops(w, threads: int, n_qtiles: int = 64) -> float:
+def oracle_exec_flops(w, threads: int, max_full: int = 4, n_qtiles: int = 64):
     """Executed-tile FLOPs of one step of ``w`` from the oracle's own tile
-    classes on ``n_qtiles`` evenly spaced q-tile rows per distinct mask."""
+    classes: every q tile of every distinct mask when the workload has at most
+    ``max_full`` distinct masks (exact), else ``n_qtiles`` evenly spaced q-tile
+    rows per distinct mask (extrapolated).  Returns (FLOPs, how)."""
     import oracle
     grid = (w.T, w.H, w.W)
     L = max(128, w.q_tile, w.kv_tile)        # the tile-major slots: padded grid in whole tiles
     n_slots = -(-oracle.padded_tokens(grid, w.unit) // L) * L
     nq = n_slots // w.q_tile
-    sample_q = np.unique(np.linspace(0, nq - 1, n_qtiles).round().astype(np.int64))
+    distinct = {tuple(sorted(s.items())) for s in w.specs}
+    exact = len(distinct) <= max_full
+    sample_q = np.arange(nq) if exact else np.unique(np.linspace(0, nq - 1, n_qtiles).round().astype(np.int64))
     counts, done = np.zeros((w.heads, 3)), {}
     for h in range(w.heads):
         key = tuple(sorted(w.specs[h].items()))
@@ -320,7 +324,9 @@ def oracle_exec_flops(w, threads: int, n_qtiles: int = 64) -> float:
             cls = fn(w.specs[h], grid, w.unit, n_slots, w.q_tile, w.kv_tile, sample_q, threads)
             done[key] = [(cls == c).sum() * nq / len(sample_q) for c in range(3)]
         counts[h] = done[key]
-    return exec_flops(w, counts) * w.B
+    how = ("from the oracle's classes of every q tile of each distinct mask" if exact else
+           f"from the oracle's classes on {len(sample_q)} evenly spaced q-tile rows per distinct mask")
+    return exec_flops(w, counts) * w.B, how
 
 
 def bench_config(w, world: int, partition: str):
@@ -338,13 +344,12 @@ def run_reference(args, w, world, rank):
         return
     import oracle
     threads = oracle.default_threads()
-    flops = oracle_exec_flops(w, threads)
+    flops, how = oracle_exec_flops(w, threads)
     R = 256
     for i in range(args.warmup):              # untimed: page in inputs, warm the caches
         oracle_sample_step(w, 16, 10_000 + i, threads)
     value, est, wall, sample = oracle_rate(w, flops, args.steps, R, threads)
-    sample += (f"; executed tiles from the oracle's classes on 64 evenly spaced q-tile rows per distinct mask; "
-               f"ms_per_step is the wall time of one sample step")
+    sample += f"; executed tiles {how}; ms_per_step is the wall time of one sample step"
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,

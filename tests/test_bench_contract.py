@@ -48,3 +48,19 @@ def test_warmup_below_three_refused():
     r = _run(["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "2"])
     assert r.returncode != 0
     assert "warmup" in r.stderr
+
+
+def test_reference_arm_flops_equal_the_oracle_goldens():
+    """The CPU arm counts executed tiles with the oracle over every q tile; on
+    the SVG workload that must equal the full-map counts stored in
+    tests/golden/full_maps.json (so both arms divide the same FLOPs)."""
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    from _helpers import full_maps, heads_of
+    w = W.svg_wan720p()
+    flops, how = bench.oracle_exec_flops(w, 8)
+    executed = sum(h["counts"][1] + h["counts"][2] for h in heads_of(full_maps()[w.name]))
+    assert "every q tile" in how
+    assert flops == 4.0 * w.D * w.q_tile * w.kv_tile * executed
