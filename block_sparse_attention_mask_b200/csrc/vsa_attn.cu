@@ -130,6 +130,7 @@ struct AttnParams {
     float* lse;
     const int32_t* list_cnt;
     const int32_t* list;
+    const int8_t* pair;                 // [heads][ceil(nE/2)]: 1 = the two blocks run as one 256-row CTA
     const int2* seg;
     const vsa_mask_spec* specs;
     const uint32_t* sbits;
@@ -366,8 +367,9 @@ __device__ __forceinline__ void mask_worker_loop(const vsa_mask_spec& m_in, cons
     }
 }
 
+// One 128-row execution block e of (batch, head) hb.
 template <int D, int BK>
-__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
+__device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
 {
     using C = Cfg<D, BK>;
     extern __shared__ uint8_t smem_raw[];
@@ -376,9 +378,6 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const vsa_dims& d = P.d;
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    const int e = blockIdx.x % d.nE;
-    const int hb = blockIdx.x / d.nE;                   // b * heads + head
     const int head = hb % d.heads;
     const long long base_row = (long long)hb * d.Nslots;
     const long long row0 = base_row + (long long)e * kRows;
@@ -884,13 +883,481 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     }
 }
 
+// ---- paired blocks: two 128-row sub-tiles per CTA ---------------------------
+//
+// Two adjacent 128-row execution blocks whose kv-tile lists hold the same kv
+// tiles (both halves of a 256-row q tile always do; 128-row q tiles do where
+// the mask repeats, e.g. inside a frame of an SVG spatial head) run in one
+// CTA, which loads every K and V tile once for both ("Sparse VideoGen ... on
+// TPU", "tile-size tuning can introduce trade-offs": how rows are grouped
+// decides the work per loaded tile).  Softmax warpgroup X owns sub-tile X
+// (rows [128 X, 128 X + 128)) with its own score buffer S_X and accumulator
+// O_X, takes its classes from its own block's list and runs every tile; the
+// two sub-tiles share the K/V ring, so the shared-memory traffic per step
+// drops by a fifth (Q 32 KB + K 32 KB + V 32 KB read, plus half the 64 KB of
+// fills, against the full fills of a single block).
+// Warps: 0..7 softmax (warpgroup X = warp / 4), 8 TMA producer (lane 0 Q and
+// K, lane 1 V), 9 MMA issuer, 10..11 idle (they keep the register split of
+// the single-block body).  MMA order per tile j: PV_0(j), QK_0(j+1), PV_1(j),
+// QK_1(j+1) after QK_0(0), QK_1(0); S_X of tile j+1 is queued behind PV_X(j),
+// so when S_X(j) is complete, O_X holds the sum up to tile j-1.  Boundary
+// bits: single-box tiles from the tile's first run descriptor, frame-0-first
+// heads by runs of frames, other tiles run by run, all in the softmax threads.
+// TMEM columns: S_0 [0,BK), S_1 [BK,2BK), O_0 [2BK,2BK+D), O_1 [2BK+D,2BK+2D).
+template <int D, int BK>
+struct PairCfg {
+    static constexpr int KV_BYTES = BK * D * 2;
+    static constexpr int QH_BYTES = kRows * D * 2;          // one 128-row sub-tile
+    static constexpr int REGS_SOFTMAX = BK == 128 ? 208 : 176;
+    static constexpr int REGS_OTHER = 3 * kRegsLaunch - 2 * REGS_SOFTMAX;
+    static constexpr int RING_BYTES = 192 * 1024 - 2 * QH_BYTES;
+    static constexpr int STAGES_V = (RING_BYTES / KV_BYTES) / 2 > 4 ? 4 : (RING_BYTES / KV_BYTES) / 2;
+    static constexpr int STAGES_K = (RING_BYTES / KV_BYTES - STAGES_V) > 4 ? 4 : (RING_BYTES / KV_BYTES - STAGES_V);
+    static_assert(STAGES_V >= 2 && STAGES_K >= 2, "shared-memory ring");
+    static constexpr int COL_S0 = 0;
+    static constexpr int COL_S1 = BK;
+    static constexpr int COL_O0 = 2 * BK;
+    static constexpr int COL_O1 = 2 * BK + D;
+    static constexpr int COLS_USED = 2 * BK + 2 * D;
+    static constexpr int TMEM_COLS = COLS_USED <= 256 ? 256 : 512;
+    static_assert(COLS_USED <= 512, "TMEM budget");
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * QH_BYTES;
+    static constexpr int OFF_V = OFF_K + STAGES_K * KV_BYTES;
+    static constexpr int OFF_ROWCTX = OFF_V + STAGES_V * KV_BYTES;
+    static constexpr int OFF_BAR = OFF_ROWCTX + 2 * kRows * (int)sizeof(vsa_row_ctx);
+    // barriers: k_full[SK], k_empty[SK], v_full[SV], v_empty[SV], q_full,
+    //           s_full[2], p_full[2], pv_done[2], mma_drain
+    static constexpr int NBAR = 2 * STAGES_K + 2 * STAGES_V + 8;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int OFF_TAB = (OFF_MISC + 20 + 15) / 16 * 16;
+    static constexpr uint32_t IDESC_QK = Cfg<D, BK>::IDESC_QK;
+    static constexpr uint32_t IDESC_PV = Cfg<D, BK>::IDESC_PV;
+};
+
+// Keep bits of query row q for a kv tile made of several boxes (a tile longer
+// than a unit): run by run from the tile's run descriptors (bw keys sharing t
+// and h each; bw divides 32, so no run straddles a 32-key word).
+template <int BK>
+__device__ __forceinline__ void multi_row_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                               const uint32_t* stab, const uint32_t* ttab,
+                                               const int2* __restrict__ seg, int kv, uint32_t (&words)[BK / 32])
+{
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) words[wi] = 0u;
+    const int2* sg = seg + (size_t)kv * d.nseg;
+    uint32_t acc = 0;
+    for (int r = 0; r < d.nseg; ++r) {
+        const int2 v = __ldg(sg + r);
+        const uint32_t b = vsa_run_bits(m, d, q, stab, ttab, v.x & 0xFFFF, v.x >> 16, v.y & 0xFFFF, v.y >> 16);
+        const int col = r * d.bw;
+        acc |= b << (col & 31);
+        if (((col + d.bw) & 31) == 0) {
+#pragma unroll
+            for (int wi = 0; wi < BK / 32; ++wi) words[wi] = (col >> 5) == wi ? acc : words[wi];
+            acc = 0;
+        }
+    }
+}
+
+// The execution blocks 2 e2 and 2 e2 + 1 of (batch, head) hb, whose lists
+// hold the same kv tiles in the same order, as one 256-row CTA.
+template <int D, int BK>
+__device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
+{
+    using C = PairCfg<D, BK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+
+    const vsa_dims& d = P.d;
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    const int head = hb % d.heads;
+    const long long base_row = (long long)hb * d.Nslots;
+    const long long row0 = base_row + (long long)e2 * 2 * kRows;
+    // the two blocks' lists name the same kv tiles: the copies follow the
+    // first, each sub-tile takes its classes from its own
+    const int list_idx = head * d.nE + 2 * e2;
+    const int cnt = P.list_cnt[list_idx];
+    const int32_t* entries = P.list + (size_t)list_idx * d.nK;
+
+    const uint32_t s_base = smem_addr(smem);
+    const uint32_t bar0 = s_base + C::OFF_BAR;
+    auto BAR_KF = [&](int s) { return bar0 + 8u * s; };
+    auto BAR_KE = [&](int s) { return bar0 + 8u * (C::STAGES_K + s); };
+    auto BAR_VF = [&](int s) { return bar0 + 8u * (2 * C::STAGES_K + s); };
+    auto BAR_VE = [&](int s) { return bar0 + 8u * (2 * C::STAGES_K + C::STAGES_V + s); };
+    constexpr int B1 = 2 * C::STAGES_K + 2 * C::STAGES_V;
+    const uint32_t BAR_QF = bar0 + 8u * B1;
+    auto BAR_SF = [&](int x) { return bar0 + 8u * (B1 + 1 + x); };
+    auto BAR_PF = [&](int x) { return bar0 + 8u * (B1 + 3 + x); };
+    auto BAR_PV = [&](int x) { return bar0 + 8u * (B1 + 5 + x); };
+    const uint32_t BAR_DR = bar0 + 8u * (B1 + 7);
+    vsa_row_ctx* rowctx = (vsa_row_ctx*)(smem + C::OFF_ROWCTX);
+    uint32_t* tmem_slot = (uint32_t*)(smem + C::OFF_MISC);
+    volatile int* abort_flag = (volatile int*)(smem + C::OFF_MISC + 4);
+    volatile int* issued = (volatile int*)(smem + C::OFF_MISC + 8);
+    uint32_t* stab = (uint32_t*)(smem + C::OFF_TAB);
+    uint32_t* ttab = stab + P.tab_words_s;
+    const Ctl ctl{abort_flag, P.status};
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES_K; ++s) {
+            mbar_init(BAR_KF(s), 1);
+            mbar_init(BAR_KE(s), 1);
+        }
+        for (int s = 0; s < C::STAGES_V; ++s) {
+            mbar_init(BAR_VF(s), 1);
+            mbar_init(BAR_VE(s), 1);
+        }
+        mbar_init(BAR_QF, 1);
+        mbar_init(BAR_DR, 1);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(BAR_SF(x), 1);
+            mbar_init(BAR_PF(x), 4);                    // the four warps of warpgroup x
+            mbar_init(BAR_PV(x), 1);
+        }
+        *abort_flag = 0;
+        issued[0] = issued[1] = issued[2] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == kMmaWarp) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(tmem_slot)),
+                     "r"((uint32_t)C::TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == kProducerWarp) {
+        // ---------------- TMA producer: lane 0 Q and K, lane 1 V ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+        if (lane == 0 && cnt > 0) {
+            mbar_expect_tx(BAR_QF, 2 * C::QH_BYTES);
+            for (int x = 0; x < 2; ++x)
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(s_base + C::OFF_Q + x * C::QH_BYTES + c * kRows * 128, &P.tm_q, c * 64,
+                                (int)(row0 + x * kRows), BAR_QF);
+            int nk = 0;
+            for (int j = 0; j < cnt; ++j, nk = j) {
+                const int st = j % C::STAGES_K;
+                if (j >= C::STAGES_K && !mbar_wait(BAR_KE(st), (uint32_t)(j / C::STAGES_K - 1) & 1, ctl)) break;
+                const int krow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
+                mbar_expect_tx(BAR_KF(st), C::KV_BYTES);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(s_base + C::OFF_K + st * C::KV_BYTES + c * BK * 128, &P.tm_k, c * 64, krow,
+                                BAR_KF(st));
+            }
+            issued[0] = nk;
+        } else if (lane == 1 && cnt > 0) {
+            int nv = 0;
+            for (int j = 0; j < cnt; ++j, nv = j) {
+                const int st = j % C::STAGES_V;
+                if (j >= C::STAGES_V && !mbar_wait(BAR_VE(st), (uint32_t)(j / C::STAGES_V - 1) & 1, ctl)) break;
+                const int vrow = (int)(base_row + (long long)VSA_ENTRY_KV(__ldg(entries + j)) * BK);
+                mbar_expect_tx(BAR_VF(st), C::KV_BYTES);
+                for (int c = 0; c < D / 64; ++c)
+                    tma_load_2d(s_base + C::OFF_V + st * C::KV_BYTES + c * BK * 128, &P.tm_v, c * 64, vrow,
+                                BAR_VF(st));
+            }
+            issued[1] = nv;
+        }
+        __syncwarp();
+    } else if (warp == kMmaWarp) {
+        // ---------------- MMA issuer ----------------
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+        const uint32_t leader = elect_one();
+        if (cnt > 0 && mbar_wait_warp(BAR_QF, 0, ctl)) {
+            tc_fence_after();
+            const uint64_t qdesc0 = smem_desc(s_base + C::OFF_Q, 16, 1024);
+            const uint64_t kdesc0 = smem_desc(s_base + C::OFF_K, 16, 1024);
+            const uint64_t vdesc0 = smem_desc(s_base + C::OFF_V, BK * 128, 1024);
+            constexpr uint64_t kStageStep = (uint64_t)(C::KV_BYTES >> 4);
+            constexpr uint64_t kQStep = (uint64_t)(C::QH_BYTES >> 4);
+            // S_X(j) = Q_X K_j^T into S_X; K_j's stage is released after sub-tile 1's QK
+            auto issue_qk = [&](int j, int x) {
+                const int st = j % C::STAGES_K;
+                const uint32_t dS = tmem + (x ? C::COL_S1 : C::COL_S0);
+                const uint64_t kd = kdesc0 + (uint64_t)st * kStageStep;
+                const uint64_t qd = qdesc0 + (uint64_t)x * kQStep;
+                mma_ss_lead<0>(dS, qd, kd, C::IDESC_QK, leader);
+#pragma unroll
+                for (int kk = 1; kk < D / 16; ++kk)
+                    mma_ss_lead<1>(dS, qd + (uint64_t)((((kk >> 2) * (kRows * 128)) + (kk & 3) * 32) >> 4),
+                                   kd + (uint64_t)((((kk >> 2) * (BK * 128)) + (kk & 3) * 32) >> 4), C::IDESC_QK,
+                                   leader);
+                tc_commit_lead(BAR_SF(x), leader);
+                if (x == 1) tc_commit_lead(BAR_KE(st), leader);
+            };
+            bool go = mbar_wait_warp(BAR_KF(0), 0, ctl);
+            if (go) {
+                tc_fence_after();
+                issue_qk(0, 0);
+                issue_qk(0, 1);
+                if (leader) issued[2] = 1;
+            }
+            for (int j = 0; go && j < cnt; ++j) {
+                const int vs = j % C::STAGES_V;
+                if (!mbar_wait_warp(BAR_VF(vs), (uint32_t)(j / C::STAGES_V) & 1, ctl)) break;
+                if (j + 1 < cnt &&
+                    !mbar_wait_warp(BAR_KF((j + 1) % C::STAGES_K), (uint32_t)((j + 1) / C::STAGES_K) & 1, ctl))
+                    break;
+                const uint64_t vd = vdesc0 + (uint64_t)vs * kStageStep;
+                for (int x = 0; x < 2; ++x) {
+                    if (!mbar_wait_warp(BAR_PF(x), (uint32_t)j & 1, ctl)) {
+                        go = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    // O_X (+)= P_X(j) V_j, P in the first BK/2 columns of S_X
+                    const uint32_t dO = tmem + (x ? C::COL_O1 : C::COL_O0);
+                    const uint32_t aP = tmem + (x ? C::COL_S1 : C::COL_S0);
+                    if (j == 0) mma_ts_lead<0>(dO, aP, vd, C::IDESC_PV, leader);
+                    else mma_ts_lead<1>(dO, aP, vd, C::IDESC_PV, leader);
+#pragma unroll
+                    for (int kk = 1; kk < BK / 16; ++kk)
+                        mma_ts_lead<1>(dO, aP + kk * 8, vd + (uint64_t)((kk * 16 * 128) >> 4), C::IDESC_PV, leader);
+                    tc_commit_lead(BAR_PV(x), leader);
+                    if (x == 1) tc_commit_lead(BAR_VE(vs), leader);
+                    // S_X(j+1) reuses S_X: queued behind PV_X(j), so P_X(j) is read first
+                    if (j + 1 < cnt) issue_qk(j + 1, x);
+                }
+            }
+        }
+    } else if (warp >= kMaskWarp0) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(C::REGS_OTHER));
+    } else {
+        // ---------------- softmax: warpgroup X owns sub-tile X ----------------
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(C::REGS_SOFTMAX));
+        const int X = warp >> 2;
+        const int r = threadIdx.x & (kRows - 1);          // TMEM lane
+        const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + lane_off + (X ? C::COL_S1 : C::COL_S0);
+        const uint32_t tO = tmem + lane_off + (X ? C::COL_O1 : C::COL_O0);
+        const vsa_mask_spec m = P.specs[head];
+        vsa_mask_spec mb = m;                             // a rounded head only masks padding
+        if (m.tile_round) {
+            mb.kind = VSA_MASK_FULL;
+            mb.sink = 0;
+        }
+        if (mb.kind == VSA_MASK_STRIPE) {
+            const uint32_t* src = P.sbits + (size_t)head * d.sbits_words;
+            for (int i = threadIdx.x; i < P.tab_words_s; i += 32 * kSoftmaxWarps) stab[i] = src[i];
+            for (int i = threadIdx.x; i < P.tab_words_t; i += 32 * kSoftmaxWarps)
+                ttab[i] = vsa_stripe_tword(m, d.T, i);
+        }
+        rowctx[X * kRows + r] = vsa_row_init(d, mb, (long long)e2 * 2 * kRows + X * kRows + r);
+        asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
+        const bool f0 = m.layout == VSA_LAYOUT_FRAME0_FIRST;
+        const bool box = d.box_nh > 0 && !f0;
+        float m_run = -INFINITY;  // running max of scale*log2(e)*s (log2 units)
+        float l_run = 0.0f;
+        const float sl = P.scale_log2;
+        const unsigned long long sl2 = f2_pack(sl, sl);
+        bool ok = true;
+        const int32_t* own = entries + (size_t)X * d.nK;  // sub-tile X's list (block 2 e2 + X)
+        int ent_next = cnt > 0 ? __ldg(own) : 0;
+        for (int j = 0; j < cnt && ok; ++j) {
+            const int ent = ent_next;
+            if (j + 1 < cnt) ent_next = __ldg(own + j + 1);
+            // one class for the 128 rows of the sub-tile (q tiles of 128 or 256 rows)
+            const int cls = VSA_ENTRY_CLS(ent, 0);
+            const int kv = VSA_ENTRY_KV(ent);
+            uint32_t mw[BK / 32];
+            if (cls == VSA_TILE_BOUNDARY) {
+                const vsa_row_ctx q = rowctx[X * kRows + r];
+                if (f0) f0_row_bits<BK>(mb, d, q, kv, mw);
+                else if (box)
+                    box_row_bits_any<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                                         (long long)kv * BK < d.Npad, mw);
+                else multi_row_bits<BK>(mb, d, q, stab, ttab, P.seg, kv, mw);
+            }
+            if (!mbar_wait_warp(BAR_SF(X), (uint32_t)j & 1, ctl)) { ok = false; break; }
+            tc_fence_after();
+            float s[BK];
+            {
+                uint32_t sr[BK];
+#pragma unroll
+                for (int c = 0; c < BK / 32; ++c) tmem_ld32(tS + c * 32, sr + c * 32);
+                tmem_ld_wait();
+#pragma unroll
+                for (int c = 0; c < BK; ++c) {
+                    reg_fence(sr[c]);
+                    s[c] = __uint_as_float(sr[c]);
+                }
+            }
+            if (cls == VSA_TILE_BOUNDARY) {
+#pragma unroll
+                for (int wi = 0; wi < BK / 32; ++wi)
+#pragma unroll
+                    for (int c = 0; c < 32; ++c)
+                        if (!((mw[wi] >> c) & 1u)) s[wi * 32 + c] = -INFINITY;
+            }
+            bool need_o = false;
+            float alpha = 1.0f;
+            {
+                float mc[BK / 32];
+#pragma unroll
+                for (int g = 0; g < BK / 32; ++g) {
+                    float a = s[g * 32];
+#pragma unroll
+                    for (int c = 1; c < 31; c += 2) a = max3(a, s[g * 32 + c], s[g * 32 + c + 1]);
+                    mc[g] = fmaxf(a, s[g * 32 + 31]);
+                }
+                float mx = mc[0];
+#pragma unroll
+                for (int g = 1; g < BK / 32; ++g) mx = fmaxf(mx, mc[g]);
+                const float mxs = mx * sl;
+                if (mx != -INFINITY) {
+                    if (m_run == -INFINITY) {
+                        m_run = mxs;      // nothing accumulated for this row yet: its O row is 0
+                    } else if (mxs > m_run + kRescaleThreshold) {
+                        alpha = ex2(m_run - mxs);
+                        l_run *= alpha;
+                        m_run = mxs;
+                        need_o = true;
+                    }
+                }
+                const float mneg = (m_run == -INFINITY) ? 0.0f : -m_run;
+                const unsigned long long mneg2 = f2_pack(mneg, mneg);
+                unsigned long long acc[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+                for (int q = 0; q < BK / 32; ++q) {
+                    uint32_t pq[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int c = 32 * q + 2 * i;
+                        float x0, x1;
+                        f2_unpack(f2_fma(f2_pack(s[c], s[c + 1]), sl2, mneg2), x0, x1);
+                        const float p0 = ex2(x0);
+                        const float p1 = ex2(x1);
+                        acc[i & 3] = f2_add(acc[i & 3], f2_pack(p0, p1));
+                        pq[i] = pack_bf16(p0, p1);
+                    }
+                    tmem_st16(tS + 16 * q, pq);
+                }
+                float a0, a1, a2, a3, a4, a5, a6, a7;
+                f2_unpack(acc[0], a0, a1);
+                f2_unpack(acc[1], a2, a3);
+                f2_unpack(acc[2], a4, a5);
+                f2_unpack(acc[3], a6, a7);
+                l_run += ((a0 + a1) + (a2 + a3)) + ((a4 + a5) + (a6 + a7));
+            }
+            // S_X(j) complete implies PV_X(j-1), the last MMA into O_X, is
+            // complete (one thread's MMAs run in order), so O_X can be rescaled
+            if (__any_sync(0xFFFFFFFFu, need_o)) {
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t ov[32];
+                    tmem_ld32(tO + c * 32, ov);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        reg_fence(ov[i]);
+                        ov[i] = __float_as_uint(__uint_as_float(ov[i]) * alpha);
+                    }
+                    tmem_st32(tO + c * 32, ov);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR_PF(X));
+        }
+
+        // ---------------- epilogue: each warpgroup writes its own 128 rows ----------------
+        bool have_o = ok;
+        if (have_o && cnt > 0) have_o = mbar_wait_warp(BAR_PV(X), (uint32_t)(cnt - 1) & 1, ctl);
+        tc_fence_after();
+        have_o = have_o && !*abort_flag;
+        const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+        const long long orow = row0 + X * kRows + r;
+        uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D);
+        if (have_o && cnt > 0) {
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t ov[32];
+                tmem_ld32(tO + c * 32, ov);
+                tmem_ld_wait();
+                uint32_t pkd[16];
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                    reg_fence(ov[i]);
+                    reg_fence(ov[i + 1]);
+                    pkd[i >> 1] = pack_bf16(__uint_as_float(ov[i]) * inv, __uint_as_float(ov[i + 1]) * inv);
+                }
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    optr[c * 4 + i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) optr[i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        P.lse[orow] = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+    }
+
+    // ---------------- teardown ----------------
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag) {
+        if (warp == kProducerWarp && lane == 0 && cnt > 0) {
+            const int nk = issued[0];
+            mbar_drain(BAR_QF, 0, kDrainCycles);
+            for (int j = nk > C::STAGES_K ? nk - C::STAGES_K : 0; j < nk; ++j)
+                mbar_drain(BAR_KF(j % C::STAGES_K), (uint32_t)(j / C::STAGES_K) & 1, kDrainCycles);
+        }
+        if (warp == kProducerWarp && lane == 1) {
+            const int nv = issued[1];
+            for (int j = nv > C::STAGES_V ? nv - C::STAGES_V : 0; j < nv; ++j)
+                mbar_drain(BAR_VF(j % C::STAGES_V), (uint32_t)(j / C::STAGES_V) & 1, kDrainCycles);
+        }
+        if (warp == kMmaWarp && issued[2]) {
+            const uint32_t leader = elect_one();
+            tc_commit_lead(BAR_DR, leader);
+            if (leader) mbar_drain(BAR_DR, 0, kDrainCycles);
+            __syncwarp();
+        }
+        tc_fence_before();
+        __syncthreads();
+    }
+    if (warp == kMmaWarp) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"((uint32_t)C::TMEM_COLS)
+                     : "memory");
+    }
+}
+
+// One CTA per (batch, head, 128-row block); where the plan pairs blocks 2p
+// and 2p + 1, the even CTA runs both and the odd one returns at once.
+template <int D, int BK>
+__global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
+{
+    const vsa_dims& d = P.d;
+    const int e = blockIdx.x % d.nE;
+    const int hb = blockIdx.x / d.nE;                   // b * heads + head
+    const int head = hb % d.heads;
+    const bool paired = P.pair[(size_t)head * ((d.nE + 1) >> 1) + (e >> 1)] != 0;
+    if (!paired) attn_single<D, BK>(P, e, hb);
+    else if ((e & 1) == 0) attn_pair<D, BK>(P, e >> 1, hb);
+}
+
 // ---- host side ----------------------------------------------------------
 
 template <int D, int BK>
 int launch_attn(AttnParams& P, int B, cudaStream_t s)
 {
     using C = Cfg<D, BK>;
-    const int smem = 1024 + C::OFF_TAB + 4 * (P.tab_words_s + P.tab_words_t);
+    using PC = PairCfg<D, BK>;
+    const int smem = 1024 + (C::OFF_TAB > PC::OFF_TAB ? C::OFF_TAB : PC::OFF_TAB) +
+                     4 * (P.tab_words_s + P.tab_words_t);
     if (smem > 227 * 1024) return VSA_ERR_UNSUPPORTED;
     auto kern = attn_fwd_kernel<D, BK>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
@@ -926,6 +1393,7 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
     P.lse = lse;
     P.list_cnt = plan->d_list_cnt;
     P.list = plan->d_list;
+    P.pair = plan->d_pair;
     P.seg = plan->d_seg;
     P.specs = plan->d_specs;
     P.sbits = plan->d_sbits;

@@ -643,6 +643,36 @@ bool tile_fits_unit(int B, int U, int bh, int bw)
     return (B % hw == 0) || (B % bw == 0 && hw % B == 0) || (bw % B == 0);
 }
 
+// Execution pairs: two adjacent 128-row blocks whose kv-tile lists hold the
+// same kv tiles, in the same order, run in one attention CTA, which loads
+// each K and V tile once for both.  Blocks of 256-row q tiles always pair
+// (both carry the q tile's list); blocks of 64-row q tiles never do (a
+// 128-row block already carries two q tiles' classes).  One warp per pair.
+__global__ void pair_mode_kernel(vsa_dims d, const int32_t* __restrict__ list_cnt,
+                                 const int32_t* __restrict__ list, int8_t* __restrict__ pair)
+{
+    const int nP = (d.nE + 1) >> 1;
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)d.heads * nP) return;
+    const int head = (int)(gw / nP), pp = (int)(gw - (long long)head * nP);
+    const int e0 = 2 * pp, e1 = 2 * pp + 1;
+    int same = 0;
+    if (d.Bq == 256) {
+        same = 1;
+    } else if (d.Bq == 128 && e1 < d.nE) {
+        const int c0 = list_cnt[(size_t)head * d.nE + e0], c1 = list_cnt[(size_t)head * d.nE + e1];
+        if (c0 == c1 && c0 > 0) {
+            const int32_t* l0 = list + ((size_t)head * d.nE + e0) * d.nK;
+            const int32_t* l1 = list + ((size_t)head * d.nE + e1) * d.nK;
+            bool eq = true;
+            for (int i = lane; i < c0; i += 32) eq = eq && VSA_ENTRY_KV(l0[i]) == VSA_ENTRY_KV(l1[i]);
+            same = __all_sync(0xFFFFFFFFu, eq) ? 1 : 0;
+        }
+    }
+    if (lane == 0) pair[(size_t)head * nP + pp] = (int8_t)same;
+}
+
 unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
 
 // Tiles of at most eight boxes (every frame-0-first tile; tile-major tiles of
@@ -678,6 +708,9 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
     VSA_CUDA_TRY(cudaGetLastError());
     kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
         d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
+    VSA_CUDA_TRY(cudaGetLastError());
+    pair_mode_kernel<<<blocks_for((long long)d.heads * ((d.nE + 1) / 2) * 32, 256), 256, 0, s>>>(
+        d, p->d_list_cnt, p->d_list, p->d_pair);
     VSA_CUDA_TRY(cudaGetLastError());
     return VSA_OK;
 }
@@ -730,6 +763,7 @@ static void free_plan(vsa_plan_s* p)
     cudaFree(p->d_cand);
     cudaFree(p->d_slot2tok);
     cudaFree(p->d_tok2slot);
+    cudaFree(p->d_pair);
     delete p;
 }
 
@@ -827,6 +861,7 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     ok = ok && cudaMalloc(&p->d_map, (size_t)num_heads * d.nQ * d.nK) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_list_cnt, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_list, sizeof(int32_t) * (size_t)num_heads * d.nE * d.nK) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_pair, (size_t)num_heads * ((d.nE + 1) / 2)) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_seg, sizeof(int2) * (size_t)d.nK * d.nseg) == cudaSuccess;
     if (has_stripe)
         ok = ok && cudaMalloc(&p->d_sbits, sizeof(uint32_t) * (size_t)num_heads * d.sbits_words) ==

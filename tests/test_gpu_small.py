@@ -33,6 +33,20 @@ CASES = {
     "q256_k128_d64": ((4, 16, 32), (1, 8, 16), 256, 128, 64,
                       [S("temporal", 1, rh=2, rw=5), S("stripe", 1, Tw=1, To=0, Ts=4, Sw=40, So=16, Ss=100),
                        S("full")]),
+    # 256-row q tiles run as two 128-row sub-tiles of one CTA
+    "q256_k128_mixed": ((5, 13, 20), (1, 8, 16), 256, 128, 128,
+                        [S("spatial", 1, rt=1), S("temporal", 1, rh=2, rw=3),
+                         S("stripe", 1, Tw=2, To=1, Ts=3, Sw=20, So=5, Ss=47), S("full"),
+                         S("sta", 0, kt=3, kh=1, kw=1), S("stripe", 0, Tw=1, To=0, Ts=2, Sw=7, So=0, Ss=9)]),
+    "q256_k128_multibox": ((4, 16, 32), (1, 8, 8), 256, 128, 128,
+                           [S("spatial", 1, rt=1), S("temporal", 1, rh=1, rw=2),
+                            S("stripe", 1, Tw=1, To=0, Ts=4, Sw=40, So=16, Ss=100)]),
+    "q256_k64_frame0_rounded": ((4, 9, 11), (1, 8, 8), 256, 64, 128,
+                                [S("temporal", 1, rh=1, rw=2, layout=1), S("spatial", 0, rt=0, tile_round=1),
+                                 S("full")]),
+    "q256_token_units_tail": ((3, 7, 9), (1, 1, 1), 256, 128, 64,
+                              [S("temporal", 1, rh=1, rw=1), S("stripe", 1, Tw=1, To=1, Ts=2, Sw=3, So=2, Ss=5),
+                               S("spatial", 0, rt=0)]),
     "q128_k64_units_of_64": ((4, 16, 32), (1, 8, 8), 128, 64, 128,
                              [S("spatial", 1, rt=1), S("temporal", 1, rh=1, rw=1),
                               S("sta", 0, kt=3, kh=1, kw=3)]),
