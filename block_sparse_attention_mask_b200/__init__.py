@@ -72,6 +72,7 @@ def _load() -> ctypes.CDLL:
         "vsa_plan_perm": ([vp, vp, sz, vp], i32),
         "vsa_plan_layout_perm": ([vp, i32, vp, sz, vp], i32),
         "vsa_plan_exec_steps": ([vp, vp, sz, vp], i32),
+        "vsa_plan_exec_pairs": ([vp, vp, sz, vp], i32),
         "vsa_plan_kept_pairs": ([vp, vp, sz, vp], i32),
         "vsa_plan_destroy": ([vp], i32),
         "vsa_permute": ([vp, vp, vp, i32, i32, vp], i32),
@@ -209,6 +210,16 @@ def vsa_plan_exec_steps(plan: int, stream=None) -> np.ndarray:
     out = np.empty(info["num_heads"], dtype=np.int64)
     _check(_lib.vsa_plan_exec_steps(plan, out.ctypes.data, out.size, _stream(stream)),
            "vsa_plan_exec_steps")
+    return out
+
+
+def vsa_plan_exec_pairs(plan: int, stream=None) -> np.ndarray:
+    """[heads, n_blocks] int32: partner of a pair's leader, -1 alone, -2 in the leader's CTA."""
+    info = vsa_plan_info(plan)
+    nE = info["n_slots"] // 128
+    out = np.empty((info["num_heads"], nE), dtype=np.int32)
+    _check(_lib.vsa_plan_exec_pairs(plan, out.ctypes.data, out.size, _stream(stream)),
+           "vsa_plan_exec_pairs")
     return out
 
 
@@ -374,6 +385,9 @@ class Plan:
 
     def exec_steps(self, stream=None) -> np.ndarray:
         return vsa_plan_exec_steps(self.handle, stream)
+
+    def exec_pairs(self, stream=None) -> np.ndarray:
+        return vsa_plan_exec_pairs(self.handle, stream)
 
     def kept_pairs(self, stream=None) -> np.ndarray:
         return vsa_plan_kept_pairs(self.handle, stream)

@@ -130,7 +130,7 @@ struct AttnParams {
     float* lse;
     const int32_t* list_cnt;
     const int32_t* list;
-    const int8_t* pair;                 // [heads][ceil(nE/2)]: 1 = the two blocks run as one 256-row CTA
+    const int32_t* pair;                // [heads][nE]: partner of a pair's leader, -1 alone, -2 in the leader's CTA
     const int2* seg;
     const vsa_mask_spec* specs;
     const uint32_t* sbits;
@@ -960,10 +960,10 @@ __device__ __forceinline__ void multi_row_bits(const vsa_mask_spec& m, const vsa
     }
 }
 
-// The execution blocks 2 e2 and 2 e2 + 1 of (batch, head) hb, whose lists
-// hold the same kv tiles in the same order, as one 256-row CTA.
+// The execution blocks ea and eb of (batch, head) hb, whose lists hold the
+// same kv tiles in the same order, as one CTA of two 128-row sub-tiles.
 template <int D, int BK>
-__device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
+__device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, int hb)
 {
     using C = PairCfg<D, BK>;
     extern __shared__ uint8_t smem_raw[];
@@ -975,12 +975,13 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
 
     const int head = hb % d.heads;
     const long long base_row = (long long)hb * d.Nslots;
-    const long long row0 = base_row + (long long)e2 * 2 * kRows;
+    const long long rowa = base_row + (long long)ea * kRows, rowb = base_row + (long long)eb * kRows;
     // the two blocks' lists name the same kv tiles: the copies follow the
     // first, each sub-tile takes its classes from its own
-    const int list_idx = head * d.nE + 2 * e2;
+    const int list_idx = head * d.nE + ea;
     const int cnt = P.list_cnt[list_idx];
     const int32_t* entries = P.list + (size_t)list_idx * d.nK;
+    const int32_t* entries_b = P.list + ((size_t)head * d.nE + eb) * d.nK;
 
     const uint32_t s_base = smem_addr(smem);
     const uint32_t bar0 = s_base + C::OFF_BAR;
@@ -1043,7 +1044,7 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
             for (int x = 0; x < 2; ++x)
                 for (int c = 0; c < D / 64; ++c)
                     tma_load_2d(s_base + C::OFF_Q + x * C::QH_BYTES + c * kRows * 128, &P.tm_q, c * 64,
-                                (int)(row0 + x * kRows), BAR_QF);
+                                (int)(x ? rowb : rowa), BAR_QF);
             int nk = 0;
             for (int j = 0; j < cnt; ++j, nk = j) {
                 const int st = j % C::STAGES_K;
@@ -1152,7 +1153,7 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
             for (int i = threadIdx.x; i < P.tab_words_t; i += 32 * kSoftmaxWarps)
                 ttab[i] = vsa_stripe_tword(m, d.T, i);
         }
-        rowctx[X * kRows + r] = vsa_row_init(d, mb, (long long)e2 * 2 * kRows + X * kRows + r);
+        rowctx[X * kRows + r] = vsa_row_init(d, mb, (long long)(X ? eb : ea) * kRows + r);
         asm volatile("bar.sync 1, %0;" ::"n"(32 * kSoftmaxWarps) : "memory");
         const bool f0 = m.layout == VSA_LAYOUT_FRAME0_FIRST;
         const bool box = d.box_nh > 0 && !f0;
@@ -1161,7 +1162,7 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
         const float sl = P.scale_log2;
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
-        const int32_t* own = entries + (size_t)X * d.nK;  // sub-tile X's list (block 2 e2 + X)
+        const int32_t* own = X ? entries_b : entries;   // sub-tile X's own list
         int ent_next = cnt > 0 ? __ldg(own) : 0;
         for (int j = 0; j < cnt && ok; ++j) {
             const int ent = ent_next;
@@ -1277,7 +1278,7 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
         tc_fence_after();
         have_o = have_o && !*abort_flag;
         const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
-        const long long orow = row0 + X * kRows + r;
+        const long long orow = (X ? rowb : rowa) + r;
         uint4* optr = reinterpret_cast<uint4*>(P.o + orow * D);
         if (have_o && cnt > 0) {
 #pragma unroll
@@ -1335,8 +1336,8 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int e2, int hb)
     }
 }
 
-// One CTA per (batch, head, 128-row block); where the plan pairs blocks 2p
-// and 2p + 1, the even CTA runs both and the odd one returns at once.
+// One CTA per (batch, head, 128-row block); where the plan pairs two blocks,
+// the leader's CTA runs both and the partner's returns at once.
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
 {
@@ -1344,9 +1345,9 @@ __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_cons
     const int e = blockIdx.x % d.nE;
     const int hb = blockIdx.x / d.nE;                   // b * heads + head
     const int head = hb % d.heads;
-    const bool paired = P.pair[(size_t)head * ((d.nE + 1) >> 1) + (e >> 1)] != 0;
-    if (!paired) attn_single<D, BK>(P, e, hb);
-    else if ((e & 1) == 0) attn_pair<D, BK>(P, e >> 1, hb);
+    const int partner = P.pair[(size_t)head * d.nE + e];
+    if (partner == -1) attn_single<D, BK>(P, e, hb);
+    else if (partner >= 0) attn_pair<D, BK>(P, e, partner, hb);
 }
 
 // ---- host side ----------------------------------------------------------

@@ -43,7 +43,7 @@ struct vsa_plan_s {
     int8_t* d_map;              // [heads][nQ][nK]
     int32_t* d_list_cnt;        // [heads][nE]
     int32_t* d_list;            // [heads][nE][nK]
-    int8_t* d_pair;             // [heads][ceil(nE/2)]: 1 = blocks 2p, 2p+1 execute as one 256-row CTA
+    int32_t* d_pair;            // [heads][nE]: partner block of a pair's leader, -1 alone, -2 in its leader's CTA
     int2* d_seg;                // [nK][nseg]: x = t | h << 16, y = w0 | nvalid << 16
     uint32_t* d_sbits;          // [heads][sbits_words] stripe intra-frame offset bits
     unsigned long long* d_counts;  // [heads][3] tile totals

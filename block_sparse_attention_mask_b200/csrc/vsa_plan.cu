@@ -643,34 +643,74 @@ bool tile_fits_unit(int B, int U, int bh, int bw)
     return (B % hw == 0) || (B % bw == 0 && hw % B == 0) || (bw % B == 0);
 }
 
-// Execution pairs: two adjacent 128-row blocks whose kv-tile lists hold the
-// same kv tiles, in the same order, run in one attention CTA, which loads
-// each K and V tile once for both.  Blocks of 256-row q tiles always pair
-// (both carry the q tile's list); blocks of 64-row q tiles never do (a
-// 128-row block already carries two q tiles' classes).  One warp per pair.
-__global__ void pair_mode_kernel(vsa_dims d, const int32_t* __restrict__ list_cnt,
-                                 const int32_t* __restrict__ list, int8_t* __restrict__ pair)
+// Execution pairs: two 128-row blocks whose kv-tile lists hold the same kv
+// tiles, in the same order, run in one attention CTA, which loads each K and
+// V tile once for both.  Blocks of 256-row q tiles pair with their neighbour
+// (both carry the q tile's list); blocks of 64-row q tiles never pair (a
+// 128-row block already carries two q tiles' classes).  For 128-row q tiles
+// each head takes the partner stride that pairs more blocks: 1 (block 2i
+// with 2i + 1, e.g. inside a frame of an SVG spatial head) or one t-slab of
+// units (the same spatial unit one slab later, e.g. an SVG temporal head,
+// whose kv tiles do not depend on the query's frame).  pair[e] is the
+// partner of a leading block, -1 for a block that runs alone, -2 for a block
+// that runs in its leader's CTA.  One CTA per head.
+__global__ void pair_plan_kernel(vsa_dims d, const int32_t* __restrict__ list_cnt,
+                                 const int32_t* __restrict__ list, int32_t* __restrict__ pair)
 {
-    const int nP = (d.nE + 1) >> 1;
-    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int lane = threadIdx.x & 31;
-    if (gw >= (long long)d.heads * nP) return;
-    const int head = (int)(gw / nP), pp = (int)(gw - (long long)head * nP);
-    const int e0 = 2 * pp, e1 = 2 * pp + 1;
-    int same = 0;
+    const int head = blockIdx.x;
+    const int nE = d.nE;
+    int32_t* pr = pair + (size_t)head * nE;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    __shared__ int votes[2];
+    for (int i = threadIdx.x; i < nE; i += blockDim.x) pr[i] = -1;
+    if (threadIdx.x < 2) votes[threadIdx.x] = 0;
+    __syncthreads();
+    if (d.Bq == 64) return;
     if (d.Bq == 256) {
-        same = 1;
-    } else if (d.Bq == 128 && e1 < d.nE) {
-        const int c0 = list_cnt[(size_t)head * d.nE + e0], c1 = list_cnt[(size_t)head * d.nE + e1];
-        if (c0 == c1 && c0 > 0) {
-            const int32_t* l0 = list + ((size_t)head * d.nE + e0) * d.nK;
-            const int32_t* l1 = list + ((size_t)head * d.nE + e1) * d.nK;
-            bool eq = true;
-            for (int i = lane; i < c0; i += 32) eq = eq && VSA_ENTRY_KV(l0[i]) == VSA_ENTRY_KV(l1[i]);
-            same = __all_sync(0xFFFFFFFFu, eq) ? 1 : 0;
+        for (int e = 2 * threadIdx.x; e + 1 < nE; e += 2 * blockDim.x) {
+            pr[e] = e + 1;
+            pr[e + 1] = -2;
+        }
+        return;
+    }
+    const long long slab = (long long)d.nTh * d.nTw * d.U;       // slots of one t-slab of units
+    const int F = slab % VSA_EXEC_ROWS == 0 ? (int)(slab / VSA_EXEC_ROWS) : 0;
+    const int32_t* cnt = list_cnt + (size_t)head * nE;
+    const int32_t* lst = list + (size_t)head * nE * d.nK;
+    // warp-collective: do blocks a and b list the same kv tiles?
+    auto same = [&](int a, int b) -> bool {
+        const int ca = cnt[a];
+        if (ca == 0 || ca != cnt[b]) return false;
+        const int32_t* la = lst + (size_t)a * d.nK;
+        const int32_t* lb = lst + (size_t)b * d.nK;
+        bool eq = true;
+        for (int i = lane; i < ca; i += 32) eq = eq && VSA_ENTRY_KV(la[i]) == VSA_ENTRY_KV(lb[i]);
+        return __all_sync(0xFFFFFFFFu, eq);
+    };
+    // leader of candidate c for stride st: blocks whose index / st is even
+    auto leader = [](int c, int st) { return (c / st) * 2 * st + c % st; };
+    for (int k = 0; k < 2; ++k) {
+        const int st = k == 0 ? 1 : F;
+        if (st < 1 || (k == 1 && st == 1)) continue;
+        int n = 0;
+        for (int c = warp;; c += nw) {
+            const int ea = leader(c, st);
+            if (ea + st >= nE) break;
+            n += same(ea, ea + st) ? 1 : 0;
+        }
+        if (lane == 0 && n) atomicAdd(&votes[k], n);
+    }
+    __syncthreads();
+    const int st = (F > 1 && votes[1] > votes[0]) ? F : 1;
+    if (votes[st == 1 ? 0 : 1] == 0) return;
+    for (int c = warp;; c += nw) {
+        const int ea = leader(c, st);
+        if (ea + st >= nE) break;
+        if (same(ea, ea + st) && lane == 0) {
+            pr[ea] = ea + st;
+            pr[ea + st] = -2;
         }
     }
-    if (lane == 0) pair[(size_t)head * nP + pp] = (int8_t)same;
 }
 
 unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
@@ -709,8 +749,7 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
     kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
         d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
     VSA_CUDA_TRY(cudaGetLastError());
-    pair_mode_kernel<<<blocks_for((long long)d.heads * ((d.nE + 1) / 2) * 32, 256), 256, 0, s>>>(
-        d, p->d_list_cnt, p->d_list, p->d_pair);
+    pair_plan_kernel<<<d.heads, 256, 0, s>>>(d, p->d_list_cnt, p->d_list, p->d_pair);
     VSA_CUDA_TRY(cudaGetLastError());
     return VSA_OK;
 }
@@ -861,7 +900,7 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     ok = ok && cudaMalloc(&p->d_map, (size_t)num_heads * d.nQ * d.nK) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_list_cnt, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_list, sizeof(int32_t) * (size_t)num_heads * d.nE * d.nK) == cudaSuccess;
-    ok = ok && cudaMalloc(&p->d_pair, (size_t)num_heads * ((d.nE + 1) / 2)) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_pair, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_seg, sizeof(int2) * (size_t)d.nK * d.nseg) == cudaSuccess;
     if (has_stripe)
         ok = ok && cudaMalloc(&p->d_sbits, sizeof(uint32_t) * (size_t)num_heads * d.sbits_words) ==
@@ -966,6 +1005,16 @@ extern "C" int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n,
     if (!plan || !host_dst || n < (size_t)plan->d.heads) return VSA_ERR_INVALID_ARG;
     cudaStream_t s = (cudaStream_t)stream;
     VSA_CUDA_TRY(cudaMemcpyAsync(host_dst, plan->d_steps, sizeof(unsigned long long) * plan->d.heads,
+                                 cudaMemcpyDeviceToHost, s));
+    VSA_CUDA_TRY(cudaStreamSynchronize(s));
+    return VSA_OK;
+}
+
+extern "C" int vsa_plan_exec_pairs(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream)
+{
+    if (!plan || !host_dst || n < (size_t)plan->d.heads * plan->d.nE) return VSA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    VSA_CUDA_TRY(cudaMemcpyAsync(host_dst, plan->d_pair, sizeof(int32_t) * (size_t)plan->d.heads * plan->d.nE,
                                  cudaMemcpyDeviceToHost, s));
     VSA_CUDA_TRY(cudaStreamSynchronize(s));
     return VSA_OK;

@@ -194,6 +194,18 @@ int vsa_plan_layout_perm(vsa_plan_t plan, int layout, int32_t* host_dst, size_t 
  * head, host_dst[h]; the attention kernel runs one tensor-core tile per step. */
 int vsa_plan_exec_steps(vsa_plan_t plan, int64_t* host_dst, size_t n, void* stream);
 
+/* Synchronous: how the attention kernel groups the 128-row execution blocks,
+ * host_dst[h * n_blocks + e] (n_blocks = n_slots / 128, n >= num_heads *
+ * n_blocks): the partner block of a pair's leader, -1 for a block that runs
+ * alone, -2 for a block that runs in its leader's CTA.  Two blocks pair when
+ * their kv-tile lists hold the same kv tiles in the same order, so one CTA
+ * loads each K and V tile once for both ([SVG-TPU], "tile-size tuning can
+ * introduce trade-offs"): always the two halves of a 256-row q tile; for
+ * 128-row q tiles, per head, block 2i with 2i + 1 or a block with the one a
+ * t-slab of units later, whichever pairs more; never for 64-row q tiles.
+ * The tile map and the tile counts do not change. */
+int vsa_plan_exec_pairs(vsa_plan_t plan, int32_t* host_dst, size_t n, void* stream);
+
 /* Synchronous: kept (real query, real key) pairs per head, host_dst[h]
  * (the logical density the tile map approximates; [SVG-TPU], "logical
  * sparsity is not physical sparsity").  Evaluates the element predicate on

@@ -85,6 +85,7 @@ def test_calls_reject_null_plan_on_host():
     assert L.vsa_plan_perm(None, None, 0, None) == -1
     assert L.vsa_plan_layout_perm(None, 0, None, 0, None) == -1
     assert L.vsa_plan_exec_steps(None, None, 0, None) == -1
+    assert L.vsa_plan_exec_pairs(None, None, 0, None) == -1
     assert L.vsa_plan_destroy(None) == -1
     assert L.vsa_permute(None, None, None, 1, 128, None) == -1
     assert L.vsa_unpermute(None, None, None, 1, 128, None) == -1

@@ -196,3 +196,42 @@ def test_tile_sweep(q_tile, kv_tile):
     full, bnd = _spatial_closed_form(21, q_tile, kv_tile)
     assert counts[0][2] == full and counts[0][1] == bnd
     assert bnd * 5 == full  # boundary share of executed tiles is 1/6
+
+
+def test_execution_pairs_follow_identical_lists():
+    """How the kernel groups 128-row blocks (execution only; the map is
+    unchanged): SVG spatial heads pair neighbouring blocks inside a frame,
+    temporal heads pair a block with the same unit one frame later (their kv
+    tiles do not depend on the query's frame), and every pair's two blocks
+    list the same kv tiles in the oracle's map."""
+    import block_sparse_attention_mask_b200 as vsa
+    w = W.svg_wan720p()
+    plan = vsa.Plan(list(w.specs), (w.T, w.H, w.W), w.unit, w.q_tile, w.kv_tile)
+    try:
+        pairs = plan.exec_pairs()
+        gmap = plan.tile_map()
+    finally:
+        plan.close()
+    nE = pairs.shape[1]
+    per_frame = 30                                  # 48 x 80 padded frame / 128
+    for h in range(w.heads):
+        lead = np.nonzero(pairs[h] >= 0)[0]
+        stride = 1 if h < 5 else per_frame
+        assert (pairs[h][lead] == lead + stride).all(), h
+        assert (pairs[h][lead + stride] == -2).all()
+        n_pairs = nE // 2 if h < 5 else per_frame * (w.T // 2)
+        assert len(lead) == n_pairs, (h, len(lead))
+        for e in lead[::37]:
+            assert ((gmap[h][e] != 0) == (gmap[h][e + stride] != 0)).all()
+    # 256-row q tiles always pair their halves; 64-row q tiles never pair
+    for q, expect in ((256, True), (64, False)):
+        ws = W.scaling(5, "spatial", q, 64)
+        plan = vsa.Plan(list(ws.specs), (ws.T, ws.H, ws.W), ws.unit, ws.q_tile, ws.kv_tile)
+        try:
+            pr = plan.exec_pairs()
+        finally:
+            plan.close()
+        if expect:
+            assert (pr[:, 0::2] == np.arange(1, pr.shape[1], 2)).all() and (pr[:, 1::2] == -2).all()
+        else:
+            assert (pr == -1).all()
