@@ -653,64 +653,74 @@ bool tile_fits_unit(int B, int U, int bh, int bw)
 // units (the same spatial unit one slab later, e.g. an SVG temporal head,
 // whose kv tiles do not depend on the query's frame).  pair[e] is the
 // partner of a leading block, -1 for a block that runs alone, -2 for a block
-// that runs in its leader's CTA.  One CTA per head.
-__global__ void pair_plan_kernel(vsa_dims d, const int32_t* __restrict__ list_cnt,
-                                 const int32_t* __restrict__ list, int32_t* __restrict__ pair)
+// that runs in its leader's CTA.
+//
+// Candidate c of stride st leads with block (c / st) * 2 st + c mod st (the
+// blocks whose index / st is even) and partners with the block st later.
+
+// Blocks per t-slab of units, when whole (0 otherwise).
+__host__ __device__ inline int pair_slab(const vsa_dims& d)
 {
-    const int head = blockIdx.x;
-    const int nE = d.nE;
-    int32_t* pr = pair + (size_t)head * nE;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    __shared__ int votes[2];
-    for (int i = threadIdx.x; i < nE; i += blockDim.x) pr[i] = -1;
-    if (threadIdx.x < 2) votes[threadIdx.x] = 0;
-    __syncthreads();
-    if (d.Bq == 64) return;
+    const long long slab = (long long)d.nTh * d.nTw * d.U;
+    return slab % VSA_EXEC_ROWS == 0 ? (int)(slab / VSA_EXEC_ROWS) : 0;
+}
+
+// One warp per (head, stride, candidate): flag[head][k][c] = 1 when the two
+// blocks list the same kv tiles; votes[head][k] counts them.
+__global__ void pair_flags_kernel(vsa_dims d, const int32_t* __restrict__ list_cnt,
+                                  const int32_t* __restrict__ list, int8_t* __restrict__ flag,
+                                  int* __restrict__ votes)
+{
+    const int nC = (d.nE + 1) / 2;                     // candidates per stride (at most)
+    const long long gw = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (gw >= (long long)d.heads * 2 * nC) return;
+    const int head = (int)(gw / (2 * nC));
+    const int k = (int)(gw / nC) & 1;
+    const int c = (int)(gw % nC);
+    const int F = pair_slab(d);
+    const int st = k == 0 ? 1 : F;
+    int same = 0;
+    if (d.Bq == 128 && st >= 1 && !(k == 1 && st == 1)) {
+        const int ea = (c / st) * 2 * st + c % st, eb = ea + st;
+        if (eb < d.nE) {
+            const int ca = list_cnt[(size_t)head * d.nE + ea];
+            if (ca > 0 && ca == list_cnt[(size_t)head * d.nE + eb]) {
+                const int32_t* la = list + ((size_t)head * d.nE + ea) * d.nK;
+                const int32_t* lb = list + ((size_t)head * d.nE + eb) * d.nK;
+                bool eq = true;
+                for (int i = lane; i < ca; i += 32) eq = eq && VSA_ENTRY_KV(la[i]) == VSA_ENTRY_KV(lb[i]);
+                same = __all_sync(0xFFFFFFFFu, eq) ? 1 : 0;
+            }
+        }
+    }
+    if (lane == 0) {
+        flag[((size_t)head * 2 + k) * nC + c] = (int8_t)same;
+        if (same) atomicAdd(&votes[head * 2 + k], 1);
+    }
+}
+
+// One thread per (head, block): the partner array from the stride each head
+// takes (the one with more pairs; the neighbour on ties).
+__global__ void pair_assign_kernel(vsa_dims d, const int8_t* __restrict__ flag, const int* __restrict__ votes,
+                                   int32_t* __restrict__ pair)
+{
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= (long long)d.heads * d.nE) return;
+    const int head = (int)(i / d.nE), e = (int)(i % d.nE);
+    int v = -1;
     if (d.Bq == 256) {
-        for (int e = 2 * threadIdx.x; e + 1 < nE; e += 2 * blockDim.x) {
-            pr[e] = e + 1;
-            pr[e + 1] = -2;
-        }
-        return;
+        v = (e & 1) ? -2 : (e + 1 < d.nE ? e + 1 : -1);
+    } else if (d.Bq == 128) {
+        const int nC = (d.nE + 1) / 2;
+        const int F = pair_slab(d);
+        const int k = (F > 1 && votes[head * 2 + 1] > votes[head * 2]) ? 1 : 0;
+        const int st = k ? F : 1;
+        const int ea = ((e / st) & 1) ? e - st : e;     // the candidate's leader
+        const int c = (ea / (2 * st)) * st + ea % st;
+        if (ea + st < d.nE && flag[((size_t)head * 2 + k) * nC + c]) v = (ea == e) ? e + st : -2;
     }
-    const long long slab = (long long)d.nTh * d.nTw * d.U;       // slots of one t-slab of units
-    const int F = slab % VSA_EXEC_ROWS == 0 ? (int)(slab / VSA_EXEC_ROWS) : 0;
-    const int32_t* cnt = list_cnt + (size_t)head * nE;
-    const int32_t* lst = list + (size_t)head * nE * d.nK;
-    // warp-collective: do blocks a and b list the same kv tiles?
-    auto same = [&](int a, int b) -> bool {
-        const int ca = cnt[a];
-        if (ca == 0 || ca != cnt[b]) return false;
-        const int32_t* la = lst + (size_t)a * d.nK;
-        const int32_t* lb = lst + (size_t)b * d.nK;
-        bool eq = true;
-        for (int i = lane; i < ca; i += 32) eq = eq && VSA_ENTRY_KV(la[i]) == VSA_ENTRY_KV(lb[i]);
-        return __all_sync(0xFFFFFFFFu, eq);
-    };
-    // leader of candidate c for stride st: blocks whose index / st is even
-    auto leader = [](int c, int st) { return (c / st) * 2 * st + c % st; };
-    for (int k = 0; k < 2; ++k) {
-        const int st = k == 0 ? 1 : F;
-        if (st < 1 || (k == 1 && st == 1)) continue;
-        int n = 0;
-        for (int c = warp;; c += nw) {
-            const int ea = leader(c, st);
-            if (ea + st >= nE) break;
-            n += same(ea, ea + st) ? 1 : 0;
-        }
-        if (lane == 0 && n) atomicAdd(&votes[k], n);
-    }
-    __syncthreads();
-    const int st = (F > 1 && votes[1] > votes[0]) ? F : 1;
-    if (votes[st == 1 ? 0 : 1] == 0) return;
-    for (int c = warp;; c += nw) {
-        const int ea = leader(c, st);
-        if (ea + st >= nE) break;
-        if (same(ea, ea + st) && lane == 0) {
-            pr[ea] = ea + st;
-            pr[ea + st] = -2;
-        }
-    }
+    pair[i] = v;
 }
 
 unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
@@ -749,7 +759,15 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
     kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
         d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
     VSA_CUDA_TRY(cudaGetLastError());
-    pair_plan_kernel<<<d.heads, 256, 0, s>>>(d, p->d_list_cnt, p->d_list, p->d_pair);
+    {
+        const long long nC = (d.nE + 1) / 2;
+        VSA_CUDA_TRY(cudaMemsetAsync(p->d_pair_votes, 0, sizeof(int) * 2 * d.heads, s));
+        pair_flags_kernel<<<blocks_for((long long)d.heads * 2 * nC * 32, 256), 256, 0, s>>>(
+            d, p->d_list_cnt, p->d_list, p->d_pair_flag, p->d_pair_votes);
+        VSA_CUDA_TRY(cudaGetLastError());
+        pair_assign_kernel<<<blocks_for((long long)d.heads * d.nE, 256), 256, 0, s>>>(
+            d, p->d_pair_flag, p->d_pair_votes, p->d_pair);
+    }
     VSA_CUDA_TRY(cudaGetLastError());
     return VSA_OK;
 }
@@ -803,6 +821,8 @@ static void free_plan(vsa_plan_s* p)
     cudaFree(p->d_slot2tok);
     cudaFree(p->d_tok2slot);
     cudaFree(p->d_pair);
+    cudaFree(p->d_pair_flag);
+    cudaFree(p->d_pair_votes);
     delete p;
 }
 
@@ -901,6 +921,8 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     ok = ok && cudaMalloc(&p->d_list_cnt, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_list, sizeof(int32_t) * (size_t)num_heads * d.nE * d.nK) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_pair, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_pair_flag, (size_t)num_heads * 2 * ((d.nE + 1) / 2)) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_pair_votes, sizeof(int) * 2 * (size_t)num_heads) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_seg, sizeof(int2) * (size_t)d.nK * d.nseg) == cudaSuccess;
     if (has_stripe)
         ok = ok && cudaMalloc(&p->d_sbits, sizeof(uint32_t) * (size_t)num_heads * d.sbits_words) ==
