@@ -345,7 +345,7 @@ def run_reference(args, w, world, rank):
     import oracle
     threads = oracle.default_threads()
     flops, how = oracle_exec_flops(w, threads)
-    R = 256
+    R = 512          # the same sample size as the GPU arm's cpu_baseline
     for i in range(args.warmup):              # untimed: page in inputs, warm the caches
         oracle_sample_step(w, 16, 10_000 + i, threads)
     value, est, wall, sample = oracle_rate(w, flops, args.steps, R, threads)
