@@ -56,7 +56,7 @@ import workloads as W  # noqa: E402
 METRIC = "sparse attn fwd ms & effective TFLOPS (kept tiles) vs B200 bf16 tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # kernels launched per ABI call (claimed launch count inside the timed region)
-LAUNCHES = {"plan_build": 5, "plan_build_stripe": 6, "permute": 1, "unpermute": 1, "fwd": 1,
+LAUNCHES = {"plan_build": 6, "plan_build_stripe": 7, "permute": 1, "unpermute": 1, "fwd": 1,
             "route": 3, "apply": 1}
 ROUTE_FRAC = 0.01      # sampled share of the tokens for SVG routing
 E2E_CHUNK_HEADS = 1    # heads per chunk of the copy-overlapped host-buffer path

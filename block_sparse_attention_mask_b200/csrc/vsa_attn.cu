@@ -131,6 +131,7 @@ struct AttnParams {
     const int32_t* list_cnt;
     const int32_t* list;
     const int32_t* pair;                // [heads][nE]: partner of a pair's leader, -1 alone, -2 in the leader's CTA
+    const int32_t* order;               // [heads]: heads by decreasing executed steps
     const int2* seg;
     const vsa_mask_spec* specs;
     const uint32_t* sbits;
@@ -1337,14 +1338,18 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
 }
 
 // One CTA per (batch, head, 128-row block); where the plan pairs two blocks,
-// the leader's CTA runs both and the partner's returns at once.
+// the leader's CTA runs both and the partner's returns at once.  CTAs walk
+// the heads in the plan's order (most executed steps first, every batch of
+// a head together), so the longest CTAs start first.
 template <int D, int BK>
 __global__ void __launch_bounds__(kThreads, 1) attn_fwd_kernel(const __grid_constant__ AttnParams P)
 {
     const vsa_dims& d = P.d;
     const int e = blockIdx.x % d.nE;
-    const int hb = blockIdx.x / d.nE;                   // b * heads + head
-    const int head = hb % d.heads;
+    const int u = blockIdx.x / d.nE;                    // rank * B + b
+    const int nb = (int)(gridDim.x / d.nE) / d.heads;   // batch
+    const int head = P.order[u / nb];
+    const int hb = (u % nb) * d.heads + head;           // b * heads + head
     const int partner = P.pair[(size_t)head * d.nE + e];
     if (partner == -1) attn_single<D, BK>(P, e, hb);
     else if (partner >= 0) attn_pair<D, BK>(P, e, partner, hb);
@@ -1395,6 +1400,7 @@ extern "C" int vsa_sparse_attn_fwd(const void* q, const void* k, const void* v, 
     P.list_cnt = plan->d_list_cnt;
     P.list = plan->d_list;
     P.pair = plan->d_pair;
+    P.order = plan->d_order;
     P.seg = plan->d_seg;
     P.specs = plan->d_specs;
     P.sbits = plan->d_sbits;

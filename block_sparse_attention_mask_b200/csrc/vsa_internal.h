@@ -46,6 +46,7 @@ struct vsa_plan_s {
     int32_t* d_pair;            // [heads][nE]: partner block of a pair's leader, -1 alone, -2 in its leader's CTA
     int8_t* d_pair_flag;        // [heads][2 strides][ceil(nE/2)] candidate pairs with the same kv tiles
     int* d_pair_votes;          // [heads][2 strides] matching candidates
+    int32_t* d_order;           // [heads] attention launch order: heads by decreasing executed steps
     int2* d_seg;                // [nK][nseg]: x = t | h << 16, y = w0 | nvalid << 16
     uint32_t* d_sbits;          // [heads][sbits_words] stripe intra-frame offset bits
     unsigned long long* d_counts;  // [heads][3] tile totals

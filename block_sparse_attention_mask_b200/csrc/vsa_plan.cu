@@ -723,6 +723,22 @@ __global__ void pair_assign_kernel(vsa_dims d, const int8_t* __restrict__ flag, 
     pair[i] = v;
 }
 
+// Launch order of the attention grid: heads by decreasing executed steps
+// (ties by index), so the longest CTAs start first and the last wave holds
+// the short ones.  order[rank] = head; one thread per head.
+__global__ void head_order_kernel(int heads, const unsigned long long* __restrict__ steps, int32_t* __restrict__ order)
+{
+    const int h = blockIdx.x * blockDim.x + threadIdx.x;
+    if (h >= heads) return;
+    const unsigned long long sh = steps[h];
+    int rank = 0;
+    for (int g = 0; g < heads; ++g) {
+        const unsigned long long sg = steps[g];
+        rank += (sg > sh || (sg == sh && g < h)) ? 1 : 0;
+    }
+    order[rank] = h;
+}
+
 unsigned blocks_for(long long n, int threads) { return (unsigned)((n + threads - 1) / threads); }
 
 // Tiles of at most eight boxes (every frame-0-first tile; tile-major tiles of
@@ -767,7 +783,9 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
         VSA_CUDA_TRY(cudaGetLastError());
         pair_assign_kernel<<<blocks_for((long long)d.heads * d.nE, 256), 256, 0, s>>>(
             d, p->d_pair_flag, p->d_pair_votes, p->d_pair);
+        VSA_CUDA_TRY(cudaGetLastError());
     }
+    head_order_kernel<<<blocks_for(d.heads, 256), 256, 0, s>>>(d.heads, p->d_steps, p->d_order);
     VSA_CUDA_TRY(cudaGetLastError());
     return VSA_OK;
 }
@@ -823,6 +841,7 @@ static void free_plan(vsa_plan_s* p)
     cudaFree(p->d_pair);
     cudaFree(p->d_pair_flag);
     cudaFree(p->d_pair_votes);
+    cudaFree(p->d_order);
     delete p;
 }
 
@@ -923,6 +942,7 @@ extern "C" int vsa_plan_create(const vsa_mask_spec* specs, int num_heads, int T,
     ok = ok && cudaMalloc(&p->d_pair, sizeof(int32_t) * (size_t)num_heads * d.nE) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_pair_flag, (size_t)num_heads * 2 * ((d.nE + 1) / 2)) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_pair_votes, sizeof(int) * 2 * (size_t)num_heads) == cudaSuccess;
+    ok = ok && cudaMalloc(&p->d_order, sizeof(int32_t) * (size_t)num_heads) == cudaSuccess;
     ok = ok && cudaMalloc(&p->d_seg, sizeof(int2) * (size_t)d.nK * d.nseg) == cudaSuccess;
     if (has_stripe)
         ok = ok && cudaMalloc(&p->d_sbits, sizeof(uint32_t) * (size_t)num_heads * d.sbits_words) ==
