@@ -274,33 +274,78 @@ __device__ __forceinline__ void f0_row_bits(const vsa_mask_spec& m, const vsa_di
         }
     }
 }
+// Keep bits of query row q for a kv tile that is one box inside a unit, for
+// the masks whose kept keys in such a tile form one rectangle per t-slice:
+// full, SVG spatial, SVG temporal and STA.  In a slice every kept latent row
+// keeps the same columns (all real ones; for the temporal mask the query's w
+// window) and the kept rows are one range (all real rows; for the temporal
+// mask the query's h window), so the words come from the range and the
+// column pattern replicated every bw bits, with no per-run loop.  Same bits
+// as box_row_bits for these kinds; the frame-0 sink keeps a whole slice.
 template <int BK>
-__device__ __forceinline__ void box_row_bits_any(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
-                                                 const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
-                                                 uint32_t (&words)[BK / 32])
+__device__ __forceinline__ void rect_row_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                              int2 v, bool tile_real, uint32_t (&words)[BK / 32])
 {
-    vsa_mask_spec mk = m;
-    switch (m.kind) {
-    case VSA_MASK_FULL:
-        mk.kind = VSA_MASK_FULL;
-        box_row_bits<VSA_MASK_FULL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
-        break;
-    case VSA_MASK_SVG_SPATIAL:
-        mk.kind = VSA_MASK_SVG_SPATIAL;
-        box_row_bits<VSA_MASK_SVG_SPATIAL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
-        break;
-    case VSA_MASK_SVG_TEMPORAL:
-        mk.kind = VSA_MASK_SVG_TEMPORAL;
-        box_row_bits<VSA_MASK_SVG_TEMPORAL, BK>(mk, d, q, stab, ttab, v, tile_real, words);
-        break;
-    case VSA_MASK_STA:
-        mk.kind = VSA_MASK_STA;
-        box_row_bits<VSA_MASK_STA, BK>(mk, d, q, stab, ttab, v, tile_real, words);
-        break;
-    default:
+    const int t0 = v.x & 0xFFFF, h0 = v.x >> 16, w0 = v.y & 0xFFFF;
+    const int bw = d.bw, nh = d.box_nh;
+    const int wv = tile_real ? max(0, min(bw, d.W - w0)) : 0;
+    const uint32_t vm = vsa_low_bits(wv);
+    const uint32_t rep1 = bw >= 32 ? 1u : 0xFFFFFFFFu / ((1u << bw) - 1u);   // one bit per run of bw
+    const int hv = min(nh, d.H - h0);              // latent rows of a slice inside the grid
+    int klo = 0, khi = hv - 1;                     // the mask's own rows and columns
+    uint32_t kpat = vm;
+    bool tile_on = true;
+    if (m.kind == VSA_MASK_SVG_TEMPORAL) {
+        klo = max(klo, q.hq - m.rh - h0);
+        khi = min(khi, q.hq + m.rh - h0);
+        const int lo = max(q.wq - m.rw, w0) - w0;
+        const int hi = min(q.wq + m.rw, w0 + wv - 1) - w0;
+        kpat = (lo <= hi) ? (vsa_low_bits(hi - lo + 1) << lo) : 0u;
+    } else if (m.kind == VSA_MASK_STA) {
+        const int ut = t0 / d.bt, uh = h0 / d.bh, uw = w0 / d.bw;
+        tile_on = ut >= q.sta_t && ut < q.sta_t + q.kk_t && uh >= q.sta_h && uh < q.sta_h + q.kk_h &&
+                  uw >= q.sta_w && uw < q.sta_w + q.kk_w;
+    }
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) words[wi] = 0u;
+    const int ns = d.nseg / nh;                    // t-slices of the tile
+    for (int sl = 0; sl < ns; ++sl) {
+        const int tt = t0 + sl;
+        int lo = 0, hi = hv - 1;
+        uint32_t pat = vm;
+        if (!(m.sink && tt == 0)) {
+            if (m.kind == VSA_MASK_SVG_TEMPORAL) {
+                lo = klo;
+                hi = khi;
+                pat = kpat;
+            }
+            const bool on = m.kind == VSA_MASK_SVG_SPATIAL ? vsa_iabs(tt - q.tq) <= m.rt : tile_on;
+            if (!on) hi = -1;
+        }
+        if (!q.real || tt >= d.T) hi = -1;
+        const int a = (sl * nh + lo) * bw, b = (sl * nh + hi + 1) * bw;    // bit range of the kept runs
+        const uint32_t rep = pat * rep1;
+#pragma unroll
+        for (int wi = 0; wi < BK / 32; ++wi) {
+            const int x0 = max(a, 32 * wi), x1 = min(b, 32 * wi + 32);
+            if (x0 < x1) words[wi] |= (vsa_low_bits(x1 - x0) << (x0 - 32 * wi)) & rep;
+        }
+    }
+}
+
+// Keep bits of a single-box boundary tile: the stripe mask run by run, the
+// others as a rectangle per slice.
+template <int BK>
+__device__ __forceinline__ void box_tile_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                              const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
+                                              uint32_t (&words)[BK / 32])
+{
+    if (m.kind == VSA_MASK_STRIPE) {
+        vsa_mask_spec mk = m;
         mk.kind = VSA_MASK_STRIPE;
         box_row_bits<VSA_MASK_STRIPE, BK>(mk, d, q, stab, ttab, v, tile_real, words);
-        break;
+    } else {
+        rect_row_bits<BK>(m, d, q, v, tile_real, words);
     }
 }
 
@@ -665,8 +710,8 @@ __device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
             if (bnd && box) {
                 const int kv = VSA_ENTRY_KV(ent);
                 const vsa_row_ctx q = rowctx[row];
-                box_row_bits_any<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
-                                     (long long)kv * BK < d.Npad, mw);
+                box_tile_bits<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                                  (long long)kv * BK < d.Npad, mw);
             }
             if (bnd && f0) {
                 const vsa_row_ctx q = rowctx[row];
@@ -1176,8 +1221,8 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
                 const vsa_row_ctx q = rowctx[X * kRows + r];
                 if (f0) f0_row_bits<BK>(mb, d, q, kv, mw);
                 else if (box)
-                    box_row_bits_any<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
-                                         (long long)kv * BK < d.Npad, mw);
+                    box_tile_bits<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                                      (long long)kv * BK < d.Npad, mw);
                 else multi_row_bits<BK>(mb, d, q, stab, ttab, P.seg, kv, mw);
             }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)j & 1, ctl)) { ok = false; break; }
