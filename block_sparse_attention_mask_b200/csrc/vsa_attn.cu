@@ -1209,21 +1209,22 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
         const unsigned long long sl2 = f2_pack(sl, sl);
         bool ok = true;
         const int32_t* own = X ? entries_b : entries;   // sub-tile X's own list
+        const vsa_row_ctx qrow = rowctx[X * kRows + r];   // the row's mask context, kept in registers
         int ent_next = cnt > 0 ? __ldg(own) : 0;
+        // first run descriptor of the next tile, loaded a tile ahead
+        int2 v_next = (box && cnt > 0) ? __ldg(P.seg + (size_t)VSA_ENTRY_KV(ent_next) * d.nseg) : make_int2(0, 0);
         for (int j = 0; j < cnt && ok; ++j) {
             const int ent = ent_next;
+            const int2 v_cur = v_next;
             if (j + 1 < cnt) ent_next = __ldg(own + j + 1);
             // one class for the 128 rows of the sub-tile (q tiles of 128 or 256 rows)
             const int cls = VSA_ENTRY_CLS(ent, 0);
             const int kv = VSA_ENTRY_KV(ent);
             uint32_t mw[BK / 32];
             if (cls == VSA_TILE_BOUNDARY) {
-                const vsa_row_ctx q = rowctx[X * kRows + r];
-                if (f0) f0_row_bits<BK>(mb, d, q, kv, mw);
-                else if (box)
-                    box_tile_bits<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
-                                      (long long)kv * BK < d.Npad, mw);
-                else multi_row_bits<BK>(mb, d, q, stab, ttab, P.seg, kv, mw);
+                if (f0) f0_row_bits<BK>(mb, d, qrow, kv, mw);
+                else if (box) box_tile_bits<BK>(mb, d, qrow, stab, ttab, v_cur, (long long)kv * BK < d.Npad, mw);
+                else multi_row_bits<BK>(mb, d, qrow, stab, ttab, P.seg, kv, mw);
             }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)j & 1, ctl)) { ok = false; break; }
             tc_fence_after();
@@ -1316,6 +1317,7 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(BAR_PF(X));
+            if (box && j + 1 < cnt) v_next = __ldg(P.seg + (size_t)VSA_ENTRY_KV(ent_next) * d.nseg);
         }
 
         // ---------------- epilogue: each warpgroup writes its own 128 rows ----------------
