@@ -694,6 +694,7 @@ __device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
                 }
             }
         }
+        const vsa_row_ctx qrow = rowctx[row];             // the row's mask context, kept in registers
         int ent_next = cnt > 0 ? __ldg(entries) : 0;
         int kb = 0;                                       // boundary tiles of the list so far
         for (int j = 0; j < cnt && ok; ++j) {
@@ -709,14 +710,10 @@ __device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
             uint32_t mw[BK / 32];
             if (bnd && box) {
                 const int kv = VSA_ENTRY_KV(ent);
-                const vsa_row_ctx q = rowctx[row];
-                box_tile_bits<BK>(mb, d, q, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                box_tile_bits<BK>(mb, d, qrow, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
                                   (long long)kv * BK < d.Npad, mw);
             }
-            if (bnd && f0) {
-                const vsa_row_ctx q = rowctx[row];
-                f0_row_bits<BK>(mb, d, q, VSA_ENTRY_KV(ent), mw);
-            }
+            if (bnd && f0) f0_row_bits<BK>(mb, d, qrow, VSA_ENTRY_KV(ent), mw);
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
             tc_fence_after();
             float s[BK];
