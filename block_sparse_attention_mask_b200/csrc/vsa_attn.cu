@@ -333,6 +333,20 @@ __device__ __forceinline__ void rect_row_bits(const vsa_mask_spec& m, const vsa_
     }
 }
 
+// Key of a single-box tile's keep bits for one query row: the tile's first
+// run descriptor (x = t | h << 16), with the frame reduced to what the mask
+// reads of it when the tile is one t-slice: full and SVG temporal masks see
+// the key's frame only as frame 0 (the sink) or past the grid.  Tiles with
+// equal keys have equal bits, so a row reuses the previous tile's bits while
+// the key stays the same (kv lists visit all frames of a unit position in a
+// row).
+__device__ __forceinline__ int bits_key_x(const vsa_mask_spec& m, const vsa_dims& d, int x)
+{
+    if (d.nseg != d.box_nh || (m.kind != VSA_MASK_SVG_TEMPORAL && m.kind != VSA_MASK_FULL)) return x;
+    const int t = x & 0xFFFF;
+    return (x & ~0xFFFF) | (t == 0 ? 0 : t < d.T ? 1 : 2);
+}
+
 // Keep bits of a single-box boundary tile: the stripe mask run by run, the
 // others as a rectangle per slice.
 template <int BK>
@@ -1210,6 +1224,8 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
         int ent_next = cnt > 0 ? __ldg(own) : 0;
         // first run descriptor of the next tile, loaded a tile ahead
         int2 v_next = (box && cnt > 0) ? __ldg(P.seg + (size_t)VSA_ENTRY_KV(ent_next) * d.nseg) : make_int2(0, 0);
+        uint32_t cw[BK / 32];                             // keep bits of the last single-box boundary tile
+        int ck_x = -1, ck_y = -1;                         // and their key (no descriptor has x = -1)
         for (int j = 0; j < cnt && ok; ++j) {
             const int ent = ent_next;
             const int2 v_cur = v_next;
@@ -1219,9 +1235,20 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
             const int kv = VSA_ENTRY_KV(ent);
             uint32_t mw[BK / 32];
             if (cls == VSA_TILE_BOUNDARY) {
-                if (f0) f0_row_bits<BK>(mb, d, qrow, kv, mw);
-                else if (box) box_tile_bits<BK>(mb, d, qrow, stab, ttab, v_cur, (long long)kv * BK < d.Npad, mw);
-                else multi_row_bits<BK>(mb, d, qrow, stab, ttab, P.seg, kv, mw);
+                if (f0) {
+                    f0_row_bits<BK>(mb, d, qrow, kv, mw);
+                } else if (box) {
+                    const int kx = bits_key_x(mb, d, v_cur.x);
+                    if (kx != ck_x || v_cur.y != ck_y) {
+                        box_tile_bits<BK>(mb, d, qrow, stab, ttab, v_cur, (long long)kv * BK < d.Npad, cw);
+                        ck_x = kx;
+                        ck_y = v_cur.y;
+                    }
+#pragma unroll
+                    for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = cw[wi];
+                } else {
+                    multi_row_bits<BK>(mb, d, qrow, stab, ttab, P.seg, kv, mw);
+                }
             }
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)j & 1, ctl)) { ok = false; break; }
             tc_fence_after();

@@ -529,10 +529,27 @@ __global__ void stripe_bits_kernel(vsa_dims d, const vsa_mask_spec* __restrict__
     sbits[(size_t)head * d.sbits_words + wd] = v;
 }
 
+// Position of the idx-th kv tile in a list of a tile-major head whose kv
+// tiles lie inside units: units spatial-position-major (all t-slabs of one
+// (h, w) unit position, then the next position), tiles of a unit in order.
+// Consecutive boundary tiles then mostly share their keep bits (a temporal
+// window does not depend on the key's frame), which the attention kernel
+// reuses.  Slots past the padded grid keep their place at the end.
+__device__ __forceinline__ int spatial_major_tile(const vsa_dims& d, int idx)
+{
+    const int tpu = d.U / d.Bk;                      // kv tiles per unit
+    const int nsu = d.nTh * d.nTw;                   // unit positions per t-slab
+    if (idx >= d.nTt * nsu * tpu) return idx;
+    const int q = idx / tpu;                         // su * nTt + slab
+    const int su = q / d.nTt, slab = q - su * d.nTt;
+    return (slab * nsu + su) * tpu + (idx - q * tpu);
+}
+
 // One warp per (head, execution block): the ordered list of kv tiles with a
 // kept pair for either 64-row half, with both halves' classes, plus tile and
-// step totals.
-__global__ void kv_list_kernel(vsa_dims d, const int8_t* __restrict__ map,
+// step totals.  Tile-major heads with kv tiles inside units list them
+// spatial-position-major (spatial_major_tile), the others in index order.
+__global__ void kv_list_kernel(vsa_dims d, const vsa_mask_spec* __restrict__ specs, const int8_t* __restrict__ map,
                                int32_t* __restrict__ list_cnt, int32_t* __restrict__ list,
                                unsigned long long* __restrict__ counts,
                                unsigned long long* __restrict__ steps)
@@ -549,10 +566,11 @@ __global__ void kv_list_kernel(vsa_dims d, const int8_t* __restrict__ map,
     const int8_t* m0 = map + ((size_t)head * d.nQ + r0) * d.nK;
     const int8_t* m1 = map + ((size_t)head * d.nQ + r1) * d.nK;
     int32_t* out = list + ((size_t)head * d.nE + e) * d.nK;
+    const bool spatial_major = specs[head].layout == VSA_LAYOUT_TILE_MAJOR && d.Bk <= d.U;
     int cnt = 0;
     unsigned c[3] = {0, 0, 0};
     for (int jb = 0; jb < d.nK; jb += 32) {
-        const int j = jb + lane;
+        const int j = (spatial_major && jb + lane < d.nK) ? spatial_major_tile(d, jb + lane) : jb + lane;
         int c0 = 0, c1 = 0;
         if (j < d.nK) {
             c0 = m0[j];
@@ -773,7 +791,7 @@ int vsa_build_plan_kernels(vsa_plan_s* p, cudaStream_t s)
     launch_tile_map(d, p->d_specs, p->has_stripe ? p->d_sbits : nullptr, p->d_map, s);
     VSA_CUDA_TRY(cudaGetLastError());
     kv_list_kernel<<<blocks_for((long long)d.heads * d.nE * 32, 256), 256, 0, s>>>(
-        d, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
+        d, p->d_specs, p->d_map, p->d_list_cnt, p->d_list, p->d_counts, p->d_steps);
     VSA_CUDA_TRY(cudaGetLastError());
     {
         const long long nC = (d.nE + 1) / 2;
