@@ -363,6 +363,82 @@ __device__ __forceinline__ void box_tile_bits(const vsa_mask_spec& m, const vsa_
     }
 }
 
+// Stripe keep bits of a single-slice tile before the frame test: run r
+// (latent row h0 + r) keeps the columns the intra-frame offset table allows.
+// The frame enters only as one bit for the whole tile (the frame-offset
+// table), so these words serve every frame of the unit position.
+template <int BK>
+__device__ __forceinline__ void stripe_win_words(const vsa_dims& d, const vsa_row_ctx& q, const uint32_t* stab, int2 v,
+                                                 bool tile_real, uint32_t (&words)[BK / 32])
+{
+    const int h0 = v.x >> 16, w0 = v.y & 0xFFFF;
+    const int bw = d.bw;
+    const int wv = tile_real ? max(0, min(bw, d.W - w0)) : 0;
+    const uint32_t vm = vsa_low_bits(wv);
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) words[wi] = 0u;
+    const int xbase = h0 * d.W + w0 - q.sq + d.H * d.W - 1;
+    uint32_t acc = 0;
+    for (int r = 0; r < d.nseg; ++r) {
+        uint32_t b = 0u;
+        if (h0 + r < d.H) {
+            const int x = xbase + r * d.W;
+            b = __funnelshift_r(stab[x >> 5], stab[(x >> 5) + 1], x & 31) & vm;
+        }
+        const int col = r * bw;
+        acc |= b << (col & 31);
+        if (((col + bw) & 31) == 0) {
+#pragma unroll
+            for (int wi = 0; wi < BK / 32; ++wi) words[wi] = (col >> 5) == wi ? acc : words[wi];
+            acc = 0;
+        }
+    }
+}
+
+// Keep bits of a single-box boundary tile for one query row, reusing the
+// words of the row's previous tile where they are the same: cw / (ck_x, ck_y)
+// hold the last computed words and their key.  Stripe tiles of one t-slice
+// cache the frame-free window words and apply the frame bit per tile (the
+// sink frame is computed whole); other masks cache by bits_key_x.
+template <int BK>
+__device__ __forceinline__ void cached_box_bits(const vsa_mask_spec& m, const vsa_dims& d, const vsa_row_ctx& q,
+                                                const uint32_t* stab, const uint32_t* ttab, int2 v, bool tile_real,
+                                                uint32_t (&cw)[BK / 32], int& ck_x, int& ck_y,
+                                                uint32_t (&mw)[BK / 32])
+{
+    if (m.kind == VSA_MASK_STRIPE && d.nseg == d.box_nh) {
+        const int t0 = v.x & 0xFFFF;
+        if (!q.real || t0 >= d.T) {
+#pragma unroll
+            for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = 0u;
+            return;
+        }
+        if (m.sink && t0 == 0) {
+            box_tile_bits<BK>(m, d, q, stab, ttab, v, tile_real, mw);
+            return;
+        }
+        const int kx = v.x | 0xFFFF;                 // the frame does not enter the window words
+        if (kx != ck_x || v.y != ck_y) {
+            stripe_win_words<BK>(d, q, stab, v, tile_real, cw);
+            ck_x = kx;
+            ck_y = v.y;
+        }
+        const int it = t0 - q.tq + d.T - 1;
+        const bool tk = (ttab[it >> 5] >> (it & 31)) & 1u;
+#pragma unroll
+        for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = tk ? cw[wi] : 0u;
+        return;
+    }
+    const int kx = bits_key_x(m, d, v.x);
+    if (kx != ck_x || v.y != ck_y) {
+        box_tile_bits<BK>(m, d, q, stab, ttab, v, tile_real, cw);
+        ck_x = kx;
+        ck_y = v.y;
+    }
+#pragma unroll
+    for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = cw[wi];
+}
+
 // Mask-worker loop for kv tiles made of several boxes (box_nh = 0),
 // specialised on the mask kind (uniform per CTA) so that no per-run branch on
 // the kind remains.  Thread t of the two mask warps writes the keep bits of
@@ -1238,14 +1314,8 @@ __device__ __forceinline__ void attn_pair(const AttnParams& P, int ea, int eb, i
                 if (f0) {
                     f0_row_bits<BK>(mb, d, qrow, kv, mw);
                 } else if (box) {
-                    const int kx = bits_key_x(mb, d, v_cur.x);
-                    if (kx != ck_x || v_cur.y != ck_y) {
-                        box_tile_bits<BK>(mb, d, qrow, stab, ttab, v_cur, (long long)kv * BK < d.Npad, cw);
-                        ck_x = kx;
-                        ck_y = v_cur.y;
-                    }
-#pragma unroll
-                    for (int wi = 0; wi < BK / 32; ++wi) mw[wi] = cw[wi];
+                    cached_box_bits<BK>(mb, d, qrow, stab, ttab, v_cur, (long long)kv * BK < d.Npad, cw, ck_x, ck_y,
+                                        mw);
                 } else {
                     multi_row_bits<BK>(mb, d, qrow, stab, ttab, P.seg, kv, mw);
                 }
