@@ -690,12 +690,13 @@ _REV = None
 
 
 def kernel_rev() -> str:
-    """Hash of the attention kernel's sources, to tie stored ncu counters to them."""
+    """Hash of the attention kernel's sources and of the plan code that orders
+    its kv lists (the order moves DRAM traffic), to tie stored ncu counters to them."""
     global _REV
     if _REV is None:
         import hashlib
         h = hashlib.sha256()
-        for f in ("vsa_attn.cu", "vsa_sm100.cuh"):
+        for f in ("vsa_attn.cu", "vsa_sm100.cuh", "vsa_plan.cu"):
             with open(os.path.join(ROOT, "block_sparse_attention_mask_b200", "csrc", f), "rb") as fh:
                 h.update(fh.read())
         _REV = h.hexdigest()[:16]
