@@ -787,6 +787,8 @@ __device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
         const vsa_row_ctx qrow = rowctx[row];             // the row's mask context, kept in registers
         int ent_next = cnt > 0 ? __ldg(entries) : 0;
         int kb = 0;                                       // boundary tiles of the list so far
+        uint32_t cw[BK / 32];                             // keep bits of the last single-box boundary tile
+        int ck_x = -1, ck_y = -1;                         // and their key
         for (int j = 0; j < cnt && ok; ++j) {
             const int ent = ent_next;
             if (j + 1 < cnt) ent_next = __ldg(entries + j + 1);
@@ -800,8 +802,8 @@ __device__ __forceinline__ void attn_single(const AttnParams& P, int e, int hb)
             uint32_t mw[BK / 32];
             if (bnd && box) {
                 const int kv = VSA_ENTRY_KV(ent);
-                box_tile_bits<BK>(mb, d, qrow, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
-                                  (long long)kv * BK < d.Npad, mw);
+                cached_box_bits<BK>(mb, d, qrow, stab, ttab, __ldg(P.seg + (size_t)kv * d.nseg),
+                                    (long long)kv * BK < d.Npad, cw, ck_x, ck_y, mw);
             }
             if (bnd && f0) f0_row_bits<BK>(mb, d, qrow, VSA_ENTRY_KV(ent), mw);
             if (!mbar_wait_warp(BAR_SF(X), (uint32_t)(j >> 1) & 1, ctl)) { ok = false; break; }
