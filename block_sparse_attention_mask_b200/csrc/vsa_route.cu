@@ -28,9 +28,9 @@
 //               queued behind PV_j, so P_j is read before it is overwritten,
 //               and QK_{j+1} runs while the softmax works on tile j.
 //   warps 0..7  softmax: thread r of warpgroup G owns sampled row r and keys
-//               [32G, 32G + 32) of every tile.  The two warpgroups exchange
-//               their partial row maxima through shared memory, so both keep
-//               the same running max; one running max (of the full row)
+//               [32G, 32G + 32) of every tile.  Both warpgroups read the
+//               whole tile's scores for the row max, so both keep the same
+//               running max with no exchange; one running max (of the full row)
 //               serves all three accumulators: p = 2^(s*scale*log2e - m) once
 //               per key, masked by the spatial and temporal keep bits into
 //               P_sp and P_tm; three running sums per warpgroup.
